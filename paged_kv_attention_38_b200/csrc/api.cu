@@ -1,0 +1,295 @@
+// C ABI of libpkv.so (declared in include/pkv.h): plan objects, the one
+// host-to-device copy of a schedule, and the launches behind pkv_run.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "../../include/pkv.h"
+#include "pkv_internal.h"
+#include "planner.h"
+
+namespace pkv {
+cudaError_t launch_prefill(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
+                           const void*, void*, float*, cudaStream_t);
+cudaError_t launch_decode(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
+                          const void*, void*, float*, cudaStream_t);
+cudaError_t launch_mla(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
+                       const void*, const void*, void*, float*, cudaStream_t);
+cudaError_t launch_merge_tasks(const LaunchGeom&, const DeviceView&, void*, float*, cudaStream_t);
+cudaError_t launch_merge_state(const float*, const float*, const float*, const float*, float*, float*, int, int,
+                               cudaStream_t);
+cudaError_t launch_merge_states(const float*, const float*, int, int, int, void*, float*, cudaStream_t);
+}  // namespace pkv
+
+using namespace pkv;
+
+struct pkv_plan {
+  Schedule sched;
+  const int32_t* kv_indices = nullptr;  // device, borrowed
+  // workspace layout (byte offsets)
+  size_t off_status = 0, off_units = 0, off_merges = 0, off_reqs = 0, off_lse = 0, off_o = 0, total = 0;
+  size_t staging_bytes = 0;
+  void* staging = nullptr;  // host copy of [status | units | merges | reqs]
+  bool staging_pinned = false;
+  DeviceView dv{};
+  bool uploaded = false;
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+pkv_status fail(pkv_status s, const std::string& msg) {
+  g_err = msg;
+  return s;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int query_num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+void layout_workspace(pkv_plan* p) {
+  const Schedule& s = p->sched;
+  size_t off = 0;
+  p->off_status = off;
+  off += 256;
+  p->off_units = off;
+  off = align256(off + s.units.size() * sizeof(WorkUnit));
+  p->off_merges = off;
+  off = align256(off + s.merges.size() * sizeof(MergeTask));
+  p->off_reqs = off;
+  off = align256(off + s.reqs.size() * sizeof(ReqInfo));
+  p->staging_bytes = off;
+  p->off_lse = off;
+  off = align256(off + (size_t)s.num_slots * s.geom.part_rows * sizeof(float));
+  p->off_o = off;
+  off = align256(off + (size_t)s.num_slots * s.geom.part_rows * s.geom.head_dim_v * sizeof(float));
+  p->total = off;
+}
+
+pkv_status create_common(const PlanInput& in, const int32_t* kv_indices, pkv_plan** out) {
+  if (!out) return fail(PKV_EINVAL, "out is NULL");
+  *out = nullptr;
+  pkv_plan* p = new (std::nothrow) pkv_plan();
+  if (!p) return fail(PKV_EINVAL, "out of host memory");
+  std::string err;
+  const int rc = build_schedule(in, &p->sched, &err);
+  if (rc != 0) {
+    delete p;
+    return fail(rc == 1 ? PKV_EINVAL : PKV_EUNSUPPORTED, err);
+  }
+  p->kv_indices = kv_indices;
+  layout_workspace(p);
+  *out = p;
+  return PKV_OK;
+}
+
+void fill_in(PlanInput& in, const int32_t* qo_indptr, const int32_t* kv_indptr, const int32_t* last, int32_t batch,
+             int32_t page_size, int32_t causal, float sm_scale, const pkv_plan_options* opts) {
+  in.qo_indptr = qo_indptr;
+  in.kv_indptr = kv_indptr;
+  in.kv_last_page_len = last;
+  in.batch = batch;
+  in.page_size = page_size;
+  in.causal = causal;
+  in.sm_scale = sm_scale;
+  in.num_sms = (opts && opts->num_sms > 0) ? opts->num_sms : query_num_sms();
+  in.disable_split_kv = opts ? opts->disable_split_kv : 0;
+  in.kv_chunk = opts ? opts->kv_chunk : 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_plan_create(const int32_t* qo_indptr, const int32_t* kv_indptr, const int32_t* kv_indices,
+                           const int32_t* kv_last_page_len, int32_t batch, int32_t num_qo_heads,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t page_size, int32_t causal,
+                           float sm_scale, const pkv_plan_options* opts, pkv_plan** out) {
+  PlanInput in{};
+  fill_in(in, qo_indptr, kv_indptr, kv_last_page_len, batch, page_size, causal, sm_scale, opts);
+  in.num_qo_heads = num_qo_heads;
+  in.num_kv_heads = num_kv_heads;
+  in.head_dim = head_dim;
+  in.head_dim_v = head_dim;
+  in.head_dim_pe = 0;
+  return create_common(in, kv_indices, out);
+}
+
+pkv_status pkv_plan_create_mla(const int32_t* qo_indptr, const int32_t* kv_indptr, const int32_t* kv_indices,
+                               const int32_t* kv_last_page_len, int32_t batch, int32_t num_heads,
+                               int32_t head_dim_ckv, int32_t head_dim_kpe, int32_t page_size, int32_t causal,
+                               float sm_scale, const pkv_plan_options* opts, pkv_plan** out) {
+  PlanInput in{};
+  fill_in(in, qo_indptr, kv_indptr, kv_last_page_len, batch, page_size, causal, sm_scale, opts);
+  in.num_qo_heads = num_heads;
+  in.num_kv_heads = 1;
+  in.head_dim = head_dim_ckv;
+  in.head_dim_v = head_dim_ckv;
+  in.head_dim_pe = head_dim_kpe;
+  if (head_dim_kpe <= 0) return fail(PKV_EUNSUPPORTED, "MLA needs head_dim_kpe > 0");
+  return create_common(in, kv_indices, out);
+}
+
+size_t pkv_plan_workspace_bytes(const pkv_plan* plan) { return plan ? plan->total : 0; }
+
+pkv_status pkv_plan_upload(pkv_plan* p, void* workspace, size_t bytes, void* stream) {
+  if (!p) return fail(PKV_EINVAL, "plan is NULL");
+  if (!workspace) return fail(PKV_EINVAL, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return fail(PKV_EINVAL, "workspace must be 256-byte aligned");
+  if (bytes < p->total) return fail(PKV_ENOSPACE, "workspace smaller than pkv_plan_workspace_bytes()");
+  if (!p->staging) {
+    if (cudaMallocHost(&p->staging, p->staging_bytes) == cudaSuccess) {
+      p->staging_pinned = true;
+    } else {
+      cudaGetLastError();
+      p->staging = std::malloc(p->staging_bytes);
+      if (!p->staging) return fail(PKV_EINVAL, "out of host memory");
+    }
+    uint8_t* h = static_cast<uint8_t*>(p->staging);
+    std::memset(h, 0, p->staging_bytes);
+    const Schedule& s = p->sched;
+    if (!s.units.empty()) std::memcpy(h + p->off_units, s.units.data(), s.units.size() * sizeof(WorkUnit));
+    if (!s.merges.empty()) std::memcpy(h + p->off_merges, s.merges.data(), s.merges.size() * sizeof(MergeTask));
+    if (!s.reqs.empty()) std::memcpy(h + p->off_reqs, s.reqs.data(), s.reqs.size() * sizeof(ReqInfo));
+  }
+  uint8_t* d = static_cast<uint8_t*>(workspace);
+  cudaError_t e = cudaMemcpyAsync(d, p->staging, p->staging_bytes, cudaMemcpyHostToDevice,
+                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("upload: ") + cudaGetErrorString(e));
+  p->dv.units = reinterpret_cast<const WorkUnit*>(d + p->off_units);
+  p->dv.merges = reinterpret_cast<const MergeTask*>(d + p->off_merges);
+  p->dv.reqs = reinterpret_cast<const ReqInfo*>(d + p->off_reqs);
+  p->dv.part_lse = reinterpret_cast<float*>(d + p->off_lse);
+  p->dv.part_o = reinterpret_cast<float*>(d + p->off_o);
+  p->dv.status = reinterpret_cast<int*>(d + p->off_status);
+  p->uploaded = true;
+  return PKV_OK;
+}
+
+pkv_status pkv_run(const pkv_plan* p, const void* q, const void* k_cache, const void* v_cache, int32_t num_pages,
+                   void* o, float* lse, void* stream) {
+  if (!p) return fail(PKV_EINVAL, "plan is NULL");
+  if (!p->uploaded) return fail(PKV_EINVAL, "plan not uploaded (call pkv_plan_upload)");
+  const Schedule& s = p->sched;
+  if (s.kind == kKindMla) return fail(PKV_EINVAL, "MLA plan: use pkv_run_mla");
+  if (s.units.empty()) return PKV_OK;
+  if (!q || !k_cache || !v_cache || !o || !p->kv_indices) return fail(PKV_EINVAL, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
+    return fail(PKV_EINVAL, "tensor pointers must be 16-byte aligned");
+  if (num_pages <= 0) return fail(PKV_EINVAL, "num_pages must be positive");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = s.kind == kKindDecode
+                      ? launch_decode(s.geom, p->dv, p->kv_indices, q, k_cache, v_cache, o, lse, st)
+                      : launch_prefill(s.geom, p->dv, p->kv_indices, q, k_cache, v_cache, o, lse, st);
+  if (e == cudaSuccess) e = launch_merge_tasks(s.geom, p->dv, o, lse, st);
+  if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return PKV_OK;
+}
+
+pkv_status pkv_run_mla(const pkv_plan* p, const void* q_nope, const void* q_pe, const void* ckv_cache,
+                       const void* kpe_cache, int32_t num_pages, void* o, float* lse, void* stream) {
+  if (!p) return fail(PKV_EINVAL, "plan is NULL");
+  if (!p->uploaded) return fail(PKV_EINVAL, "plan not uploaded (call pkv_plan_upload)");
+  const Schedule& s = p->sched;
+  if (s.kind != kKindMla) return fail(PKV_EINVAL, "not an MLA plan: use pkv_run");
+  if (s.units.empty()) return PKV_OK;
+  if (!q_nope || !q_pe || !ckv_cache || !kpe_cache || !o || !p->kv_indices)
+    return fail(PKV_EINVAL, "NULL tensor pointer");
+  if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(ckv_cache) || !aligned16(kpe_cache) || !aligned16(o))
+    return fail(PKV_EINVAL, "tensor pointers must be 16-byte aligned");
+  if (num_pages <= 0) return fail(PKV_EINVAL, "num_pages must be positive");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_mla(s.geom, p->dv, p->kv_indices, q_nope, q_pe, ckv_cache, kpe_cache, o, lse, st);
+  if (e == cudaSuccess) e = launch_merge_tasks(s.geom, p->dv, o, lse, st);
+  if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return PKV_OK;
+}
+
+pkv_status pkv_merge_state(const float* o_a, const float* lse_a, const float* o_b, const float* lse_b,
+                           float* o_out, float* lse_out, int32_t rows, int32_t dim, void* stream) {
+  if (rows < 0 || dim <= 0 || dim > 1024) return fail(PKV_EINVAL, "rows >= 0 and 0 < dim <= 1024 required");
+  if (rows > 0 && (!o_a || !lse_a || !o_b || !lse_b || !o_out || !lse_out)) return fail(PKV_EINVAL, "NULL pointer");
+  cudaError_t e = launch_merge_state(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, dim,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("merge_state: ") + cudaGetErrorString(e));
+  return PKV_OK;
+}
+
+pkv_status pkv_merge_states(const float* o_parts, const float* lse_parts, int32_t num, int32_t rows, int32_t dim,
+                            void* o_out, float* lse_out, void* stream) {
+  if (num <= 0 || rows < 0 || dim <= 0 || dim > 1024) return fail(PKV_EINVAL, "num > 0, rows >= 0, 0 < dim <= 1024");
+  if (rows > 0 && (!o_parts || !lse_parts || !o_out || !lse_out)) return fail(PKV_EINVAL, "NULL pointer");
+  cudaError_t e = launch_merge_states(o_parts, lse_parts, num, rows, dim, o_out, lse_out,
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("merge_states: ") + cudaGetErrorString(e));
+  return PKV_OK;
+}
+
+pkv_status pkv_device_status(const pkv_plan* p, void* stream, int32_t* code) {
+  if (!p || !p->uploaded) return fail(PKV_EINVAL, "plan not uploaded");
+  int32_t h = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&h, p->dv.status, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("status: ") + cudaGetErrorString(e));
+  if (code) *code = h;
+  if (h != 0) return fail(PKV_EDEVICE, "a kernel reported a device-side wait timeout");
+  return PKV_OK;
+}
+
+int64_t pkv_plan_info(const pkv_plan* p, int32_t key) {
+  if (!p) return -1;
+  const Schedule& s = p->sched;
+  switch (key) {
+    case 0: return s.kind;
+    case 1: return (int64_t)s.units.size();
+    case 2: return (int64_t)s.merges.size();
+    case 3: return s.num_slots;
+    case 4: return s.geom.part_rows;
+    case 5: return s.num_sms;
+    case 6: return s.kv_chunk;
+    default: return -1;
+  }
+}
+
+int32_t pkv_plan_work_units(const pkv_plan* p, int32_t* out, int32_t capacity) {
+  if (!p || !out || capacity <= 0) return 0;
+  const int32_t n = (int32_t)std::min<size_t>(p->sched.units.size(), (size_t)capacity);
+  std::memcpy(out, p->sched.units.data(), (size_t)n * sizeof(WorkUnit));
+  return n;
+}
+
+int32_t pkv_plan_merge_tasks(const pkv_plan* p, int32_t* out, int32_t capacity) {
+  if (!p || !out || capacity <= 0) return 0;
+  const int32_t n = (int32_t)std::min<size_t>(p->sched.merges.size(), (size_t)capacity);
+  std::memcpy(out, p->sched.merges.data(), (size_t)n * sizeof(MergeTask));
+  return n;
+}
+
+void pkv_plan_destroy(pkv_plan* p) {
+  if (!p) return;
+  if (p->staging) {
+    if (p->staging_pinned) cudaFreeHost(p->staging);  // waits for the copy that reads it
+    else std::free(p->staging);
+  }
+  delete p;
+}
+
+const char* pkv_last_error(void) { return g_err.c_str(); }
+
+const char* pkv_version(void) { return "pkv 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

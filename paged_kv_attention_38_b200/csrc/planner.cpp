@@ -1,0 +1,179 @@
+// Host planner (see planner.h).
+//
+// Query rows are packed per kv head: for request b and kv head g, packed row
+// r = t * group + i stands for token t of the request and qo head g*group + i.
+// A tile is kBlockM consecutive packed rows, so with a large group (h16/kv1) a
+// tile covers a few tokens of all heads that share one K/V stream, and every
+// K/V tile the CTA loads is reused by all of its rows.
+//
+// With causal masking (bottom-right, see pkv.h) the last token of a tile bounds
+// the keys the tile needs: keys [0, t_last + kv_len - qo_len + 1).
+#include "planner.h"
+
+#include <algorithm>
+#include <cmath>
+#include <numeric>
+
+namespace pkv {
+
+namespace {
+
+bool is_pow2(int32_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int ilog2(int32_t x) {
+  int s = 0;
+  while ((1 << s) < x) ++s;
+  return s;
+}
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+struct Tile {
+  int32_t req, kv_head, row0, rows, kv_need;
+};
+
+}  // namespace
+
+int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
+  Schedule s;
+  const bool mla = in.head_dim_pe > 0;
+  if (in.batch < 0) { *err = "batch < 0"; return 1; }
+  if (in.batch > 0 && (!in.qo_indptr || !in.kv_indptr || !in.kv_last_page_len)) {
+    *err = "NULL indptr / last_page_len"; return 1;
+  }
+  if (in.num_qo_heads <= 0 || in.num_kv_heads <= 0) { *err = "head counts must be positive"; return 1; }
+  if (in.num_qo_heads % in.num_kv_heads != 0) { *err = "num_qo_heads % num_kv_heads != 0"; return 1; }
+  if (!is_pow2(in.page_size) || in.page_size > 256) {
+    *err = "page_size must be a power of two in [1, 256]"; return 2;
+  }
+  if (!std::isfinite(in.sm_scale)) { *err = "sm_scale is not finite"; return 1; }
+  const int32_t group = in.num_qo_heads / in.num_kv_heads;
+  if (mla) {
+    if (in.num_kv_heads != 1 || in.head_dim != 512 || in.head_dim_v != 512 || in.head_dim_pe != 64) {
+      *err = "MLA supports head_dim_ckv 512, head_dim_kpe 64, one latent head"; return 2;
+    }
+    if (in.num_qo_heads > 128) { *err = "MLA supports at most 128 heads"; return 2; }
+  } else {
+    if (in.head_dim != 64 && in.head_dim != 128) { *err = "head_dim must be 64 or 128"; return 2; }
+    if (in.head_dim_v != in.head_dim) { *err = "head_dim_v must equal head_dim"; return 2; }
+    if (group > 128) { *err = "group size num_qo_heads / num_kv_heads must be <= 128"; return 2; }
+  }
+
+  // ---- validate the page table, build per-request info
+  if (in.batch > 0) {
+    if (in.qo_indptr[0] != 0 || in.kv_indptr[0] != 0) { *err = "indptr must start at 0"; return 1; }
+  }
+  s.reqs.resize(in.batch);
+  int32_t max_qo = 0;
+  for (int32_t b = 0; b < in.batch; ++b) {
+    const int32_t qo = in.qo_indptr[b + 1] - in.qo_indptr[b];
+    const int32_t np = in.kv_indptr[b + 1] - in.kv_indptr[b];
+    if (qo < 0) { *err = "qo_indptr is not non-decreasing"; return 1; }
+    if (np < 0) { *err = "kv_indptr is not non-decreasing"; return 1; }
+    const int32_t last = in.kv_last_page_len[b];
+    if (np > 0 && (last < 1 || last > in.page_size)) {
+      *err = "kv_last_page_len must be in [1, page_size] for a request with pages"; return 1;
+    }
+    const int64_t kv_len = np > 0 ? (int64_t)(np - 1) * in.page_size + last : 0;
+    if (kv_len > INT32_MAX / 2) { *err = "kv_len too large"; return 2; }
+    if ((int64_t)qo * group > INT32_MAX / 2) { *err = "qo_len * group too large"; return 2; }
+    s.reqs[b] = ReqInfo{in.qo_indptr[b], qo, (int32_t)kv_len, in.kv_indptr[b]};
+    max_qo = std::max(max_qo, qo);
+  }
+
+  // ---- kernel choice
+  if (mla) s.kind = kKindMla;
+  else if (max_qo <= 1 && group <= kDecodeRows) s.kind = kKindDecode;
+  else s.kind = kKindPrefill;
+
+  const int32_t num_sms = in.num_sms > 0 ? in.num_sms : 148;
+  s.num_sms = num_sms;
+  const int32_t tile_rows = s.kind == kKindDecode ? kDecodeRows : kBlockM;
+  // MLA tiles pack tokens x heads the same way, with a single latent "kv head".
+  const int32_t mla_tile_rows = kBlockM;
+  const int32_t rows_per_tile = s.kind == kKindMla ? mla_tile_rows : tile_rows;
+
+  // ---- tiles
+  std::vector<Tile> tiles;
+  int64_t total_cost = 0;
+  int32_t max_need = 0;
+  for (int32_t b = 0; b < in.batch; ++b) {
+    const ReqInfo& r = s.reqs[b];
+    const int64_t packed = (int64_t)r.qo_len * group;
+    for (int32_t g = 0; g < in.num_kv_heads; ++g) {
+      for (int64_t row0 = 0; row0 < packed; row0 += rows_per_tile) {
+        const int32_t rows = (int32_t)std::min<int64_t>(rows_per_tile, packed - row0);
+        const int64_t t_last = (row0 + rows - 1) / group;
+        int64_t need = r.kv_len;
+        if (in.causal) need = std::min<int64_t>(r.kv_len, std::max<int64_t>(0, t_last + r.kv_len - r.qo_len + 1));
+        tiles.push_back(Tile{b, g, (int32_t)row0, rows, (int32_t)need});
+        total_cost += need + 64;
+        max_need = std::max<int32_t>(max_need, (int32_t)need);
+      }
+    }
+  }
+
+  // ---- split-KV chunk
+  const int32_t align = s.kind == kKindDecode ? kDecodeTileN : kBlockN;
+  int64_t chunk = 0;  // 0 = no split
+  if (!in.disable_split_kv) {
+    if (in.kv_chunk > 0) {
+      chunk = round_up(in.kv_chunk, align);
+    } else if (s.kind == kKindDecode) {
+      // Decode is HBM-bound: aim for ~8 units per SM so the tail is short; a
+      // chunk below 512 keys would spend more on partial state than it saves.
+      chunk = round_up(std::max<int64_t>(512, total_cost / ((int64_t)num_sms * 8)), align);
+      chunk = std::min<int64_t>(chunk, 4096);
+    } else {
+      // Prefill: one CTA per SM at a time; split only when a single tile is
+      // longer than the average work per SM.
+      chunk = round_up(std::max<int64_t>(256, (total_cost + num_sms - 1) / num_sms), align);
+    }
+    if (chunk >= max_need) chunk = 0;
+  }
+  s.kv_chunk = (int32_t)chunk;
+
+  // ---- units and merges
+  int32_t slots = 0;
+  for (const Tile& t : tiles) {
+    if (chunk == 0 || t.kv_need <= chunk) {
+      s.units.push_back(WorkUnit{t.req, t.kv_head, t.row0, t.rows, 0, t.kv_need, -1, 0});
+      continue;
+    }
+    const int32_t n = (int32_t)((t.kv_need + chunk - 1) / chunk);
+    s.merges.push_back(MergeTask{t.req, t.kv_head, t.row0, t.rows, slots, n, 0, 0});
+    for (int32_t c = 0; c < n; ++c) {
+      const int32_t lo = (int32_t)(c * chunk);
+      const int32_t hi = (int32_t)std::min<int64_t>(t.kv_need, (int64_t)(c + 1) * chunk);
+      s.units.push_back(WorkUnit{t.req, t.kv_head, t.row0, t.rows, lo, hi, slots + c, 0});
+    }
+    slots += n;
+  }
+  s.num_slots = slots;
+
+  // Longest units first: with a non-persistent grid the hardware hands out
+  // CTAs roughly in index order, so this is a greedy longest-processing-time
+  // schedule that keeps the tail short.
+  std::stable_sort(s.units.begin(), s.units.end(), [](const WorkUnit& a, const WorkUnit& b) {
+    return (a.kv_hi - a.kv_lo) > (b.kv_hi - b.kv_lo);
+  });
+
+  LaunchGeom& gm = s.geom;
+  gm.num_qo_heads = in.num_qo_heads;
+  gm.num_kv_heads = in.num_kv_heads;
+  gm.group = group;
+  gm.head_dim = in.head_dim;
+  gm.head_dim_v = in.head_dim_v;
+  gm.head_dim_pe = in.head_dim_pe;
+  gm.page_size = in.page_size;
+  gm.page_shift = ilog2(in.page_size);
+  gm.causal = in.causal ? 1 : 0;
+  gm.sm_scale_log2 = (float)((double)in.sm_scale * 1.4426950408889634);
+  gm.part_rows = rows_per_tile;
+  gm.num_units = (int32_t)s.units.size();
+  gm.num_merge = (int32_t)s.merges.size();
+  *out = std::move(s);
+  return 0;
+}
+
+}  // namespace pkv

@@ -1,0 +1,191 @@
+"""CPU tests of the C ABI library: it loads, exports every symbol include/pkv.h
+declares, rejects malformed input with the documented status codes, and its
+host planner covers every (request, kv head, query row, key) exactly once.
+
+No GPU is needed: only host entry points are called (planning without upload).
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import paged_kv_attention_38_b200 as pkv
+from oracle import paged_ref
+from paged_kv_attention_38_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkv.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not os.path.exists(pkv.lib_path):
+        from paged_kv_attention_38_b200 import build
+        build.build()
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    lib = pkv.load_library()
+    syms = _declared_symbols()
+    assert len(syms) >= 14
+    for s in syms:
+        assert hasattr(lib, s), f"libpkv.so does not export {s}"
+    assert lib.pkv_version().decode().startswith("pkv")
+
+
+def test_no_hidden_symbol_leaks():
+    """Only the pkv_ C ABI is exported (internal C++ symbols stay hidden)."""
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", pkv.lib_path], capture_output=True, text=True).stdout
+    names = [l.split()[-1] for l in out.splitlines() if " T " in l]
+    ours = [n for n in names if n.startswith("pkv_")]
+    assert set(_declared_symbols()) <= set(ours)
+
+
+def _plan(p: W.PagedProblem, **kw):
+    kw.setdefault("num_sms", 148)
+    return pkv.plan(p.qo_indptr, p.kv_indptr, None, p.kv_last_page_len, p.num_qo_heads, p.num_kv_heads,
+                    p.head_dim, p.page_size, p.causal, p.sm_scale, upload=False, **kw)
+
+
+def _lengths_problem(qo, kv, hq=4, hk=1, d=64, ps=16, causal=True):
+    kv_indptr, kv_indices, last, _ = W.page_table(np.asarray(kv), ps, W._gen(5))
+    qo_indptr = np.concatenate([[0], np.cumsum(qo)]).astype(np.int32)
+    return W.PagedProblem("lens", qo_indptr, kv_indptr, kv_indices, last, ps, hq, hk, d, d, causal,
+                          1.0 / np.sqrt(d))
+
+
+def _check_coverage(p: W.PagedProblem, pl: pkv.Plan):
+    """Every packed row of every (request, kv head) is covered; its units' key
+    ranges partition [0, need) where need bounds the keys any row of the tile sees."""
+    G = p.num_qo_heads // p.num_kv_heads
+    units = pl.work_units()
+    merges = pl.merge_tasks()
+    rows_per = pl.info(4)
+    tiles = {}
+    for u in units:
+        req, g, row0, rows, lo, hi, part, _ = u.tolist()
+        tiles.setdefault((req, g, row0, rows), []).append((lo, hi, part))
+    kv_lens, qo_lens = p.kv_lens, p.qo_lens
+    slots_seen = set()
+    for b in range(p.batch):
+        packed = int(qo_lens[b]) * G
+        for g in range(p.num_kv_heads):
+            r = 0
+            while r < packed:
+                rows = min(rows_per, packed - r)
+                key = (b, g, r, rows)
+                assert key in tiles, f"missing tile {key}"
+                t_first, t_last = r // G, (r + rows - 1) // G
+                vis = paged_ref.visible(int(qo_lens[b]), int(kv_lens[b]), p.causal,
+                                        np.arange(t_first, t_last + 1))
+                need = int(vis.any(axis=0).nonzero()[0].max() + 1) if vis.any() else 0
+                chunks = sorted(tiles.pop(key))
+                assert chunks[0][0] == 0 and chunks[-1][1] == need
+                for (a_lo, a_hi, _), (b_lo, _, _) in zip(chunks, chunks[1:]):
+                    assert a_hi == b_lo
+                if len(chunks) == 1:
+                    assert chunks[0][2] == -1
+                else:
+                    parts = [c[2] for c in chunks]
+                    assert all(x >= 0 for x in parts)
+                    slots_seen.update(parts)
+                    m = [t for t in merges.tolist() if t[:4] == [b, g, r, rows]]
+                    assert len(m) == 1 and m[0][5] == len(chunks)
+                    assert sorted(parts) == list(range(m[0][4], m[0][4] + m[0][5]))
+                r += rows
+    assert not tiles, f"extra tiles {list(tiles)[:3]}"
+    assert len(slots_seen) == pl.info(3)
+
+
+@pytest.mark.parametrize("maker", [W.tiny_prefill, W.gqa_prefill, W.paged_decode])
+def test_planner_covers_workloads(maker):
+    p = maker()
+    _check_coverage(p, _plan(p))
+
+
+@pytest.mark.parametrize("chunk", [128, 256, 1000])
+def test_planner_forced_split(chunk):
+    p = _lengths_problem([40, 1, 300], [40, 1300, 300], hq=8, hk=2)
+    pl = _plan(p, kv_chunk=chunk)
+    _check_coverage(p, pl)
+    assert pl.num_merges > 0
+
+
+def test_planner_disable_split_kv():
+    p = _lengths_problem([1] * 4, [10000, 20000, 5, 7], hq=8, hk=2, ps=16, causal=False)
+    pl = _plan(p, disable_split_kv=True)
+    assert pl.num_merges == 0 and pl.kind == pkv.KIND_DECODE
+    _check_coverage(p, pl)
+    pl2 = _plan(p)
+    assert pl2.num_merges > 0
+    _check_coverage(p, pl2)
+
+
+def test_planner_edge_cases():
+    # empty request, qo_len > kv_len (rows with no key), qo_len = 0
+    p = _lengths_problem([5, 0, 9, 3], [0, 4, 4, 3], hq=4, hk=2, ps=2)
+    pl = _plan(p)
+    _check_coverage(p, pl)
+    # empty batch
+    p0 = _lengths_problem([], [], hq=4, hk=1)
+    pl0 = _plan(p0)
+    assert pl0.num_units == 0
+
+
+def test_planner_kinds():
+    assert _plan(W.paged_decode()).kind == pkv.KIND_DECODE
+    assert _plan(W.gqa_prefill()).kind == pkv.KIND_PREFILL
+    m = W.mla_prefill()
+    pl = pkv.plan_mla(m.qo_indptr, m.kv_indptr, None, m.kv_last_page_len, 16, 512, 64, 1, True,
+                      m.sm_scale, upload=False, num_sms=148)
+    assert pl.kind == pkv.KIND_MLA
+
+
+def test_longest_units_first():
+    pl = _plan(W.gqa_prefill())
+    u = pl.work_units()
+    lens = u[:, 5] - u[:, 4]
+    assert np.all(np.diff(lens) <= 0)
+
+
+@pytest.mark.parametrize("mutate,status", [
+    (lambda a: a["qo"].__setitem__(1, -3), pkv.PKV_EINVAL),            # qo_indptr decreasing
+    (lambda a: a["kv"].__setitem__(0, 1), pkv.PKV_EINVAL),             # kv_indptr not starting at 0
+    (lambda a: a["last"].__setitem__(0, 0), pkv.PKV_EINVAL),           # last_page_len 0 with pages
+    (lambda a: a["last"].__setitem__(0, 17), pkv.PKV_EINVAL),          # last_page_len > page_size
+    (lambda a: a.__setitem__("ps", 24), pkv.PKV_EUNSUPPORTED),         # page size not a power of two
+    (lambda a: a.__setitem__("d", 96), pkv.PKV_EUNSUPPORTED),          # unsupported head_dim
+    (lambda a: a.__setitem__("hk", 3), pkv.PKV_EINVAL),                # hq % hk != 0
+    (lambda a: a.__setitem__("scale", float("nan")), pkv.PKV_EINVAL),  # sm_scale not finite
+])
+def test_error_codes(mutate, status):
+    a = dict(qo=np.array([0, 5, 9], np.int32), kv=np.array([0, 1, 2], np.int32),
+             last=np.array([5, 4], np.int32), ps=16, d=64, hk=1, scale=0.125)
+    mutate(a)
+    with pytest.raises(pkv.PkvError) as e:
+        pkv.plan(a["qo"], a["kv"], None, a["last"], 4, a["hk"], a["d"], a["ps"], True, a["scale"],
+                 upload=False, num_sms=148)
+    assert e.value.status == status
+    assert len(pkv.load_library().pkv_last_error()) > 0
+
+
+def test_upload_rejects_bad_workspace():
+    lib = pkv.load_library()
+    p = _lengths_problem([5], [5])
+    pl = _plan(p)
+    assert lib.pkv_plan_upload(pl.handle, None, 0, None) == pkv.PKV_EINVAL
+    assert lib.pkv_plan_upload(pl.handle, 256, 1, None) == pkv.PKV_ENOSPACE
+    assert lib.pkv_plan_upload(pl.handle, 257, 1 << 20, None) == pkv.PKV_EINVAL
+    # run before upload is refused before any launch
+    assert lib.pkv_run(pl.handle, 16, 16, 16, 1, 16, 16, None) == pkv.PKV_EINVAL
+    assert lib.pkv_merge_state(None, None, None, None, None, None, 4, 0, None) == pkv.PKV_EINVAL
+    assert lib.pkv_merge_states(None, None, 0, 4, 8, None, None, None) == pkv.PKV_EINVAL

@@ -1,0 +1,238 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Tolerances (stated numbers for this path): bf16 O elementwise
+|o - ref| <= 1e-2 + 1e-2 |ref|; fp32 base-2 LSE |lse - ref| <= 1e-3; rows that
+see no key must give O = 0 and LSE = -inf exactly.
+"""
+import math
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_attention_38_b200 as pkv
+from paged_kv_attention_38_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+ATOL_O, RTOL_O, ATOL_LSE = 1e-2, 1e-2, 1e-3
+
+
+def assert_parity(o, lse, o_ref, lse_ref, what=""):
+    o = o.float().cpu().double().numpy() if hasattr(o, "cpu") else o
+    lse = lse.float().cpu().double().numpy() if hasattr(lse, "cpu") else lse
+    assert o.shape == o_ref.shape, (o.shape, o_ref.shape)
+    assert np.all(np.isfinite(o)), f"{what}: non-finite O"
+    err = np.abs(o - o_ref)
+    bad = err > ATOL_O + RTOL_O * np.abs(o_ref)
+    assert not bad.any(), (f"{what}: O mismatch at {np.argwhere(bad)[:5].tolist()}, max abs err "
+                           f"{err.max():.3e}, ref there {o_ref[bad][:3]}")
+    ninf_ref = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), ninf_ref), f"{what}: -inf LSE rows differ"
+    fin = ~ninf_ref
+    lerr = np.abs(lse[fin] - lse_ref[fin]) if fin.any() else np.zeros(1)
+    assert lerr.max() <= ATOL_LSE, f"{what}: LSE max abs err {lerr.max():.3e}"
+
+
+def to_dev(p: W.PagedProblem):
+    d = {}
+    for name in ("q", "k_cache", "v_cache", "q_nope", "q_pe", "ckv_cache", "kpe_cache"):
+        t = getattr(p, name)
+        if t is not None:
+            d[name] = t.cuda()
+    d["kv_indices"] = torch.from_numpy(p.kv_indices.astype(np.int32)).cuda()
+    return d
+
+
+def gpu_run(p: W.PagedProblem, **plan_kw):
+    d = to_dev(p)
+    pl = pkv.plan(p.qo_indptr, p.kv_indptr, d["kv_indices"], p.kv_last_page_len, p.num_qo_heads,
+                  p.num_kv_heads, p.head_dim, p.page_size, p.causal, p.sm_scale, **plan_kw)
+    o, lse = pkv.run(pl, d["q"], d["k_cache"], d["v_cache"])
+    torch.cuda.synchronize()
+    assert pkv.device_status(pl) == 0
+    return o, lse, pl
+
+
+def oracle_run(p: W.PagedProblem):
+    return oracle.paged_attention(p.q, p.k_cache, p.v_cache, p.qo_indptr, p.kv_indptr, p.kv_indices,
+                                  p.kv_last_page_len, p.page_size, p.causal, p.sm_scale)
+
+
+# --------------------------------------------------------------------------- prefill
+
+def test_tiny_prefill():
+    p = W.tiny_prefill()
+    o, lse, pl = gpu_run(p)
+    assert pl.kind == pkv.KIND_PREFILL
+    assert_parity(o, lse, *oracle_run(p), what="tiny")
+
+
+SWEEP = [
+    # qo_lens, kv_lens, hq, hk, d, page, causal
+    ([1, 127, 128, 129, 300], [1, 127, 128, 129, 300], 4, 4, 64, 16, True),
+    ([200, 33], [200, 33], 16, 1, 128, 64, True),
+    ([70, 250], [70, 250], 8, 2, 128, 1, True),
+    ([64, 190], [64, 190], 4, 1, 128, 2, True),
+    ([37, 100], [137, 400], 4, 2, 128, 16, True),     # chunked prefill: qo < kv (bottom-right)
+    ([90, 5], [60, 5], 2, 1, 64, 8, True),            # qo > kv: first rows see no key
+    ([50, 0, 80], [50, 30, 0], 4, 1, 64, 4, True),    # a request with no queries, one with no keys
+    ([45, 160], [300, 160], 8, 8, 128, 32, False),    # non-causal MHA
+    ([130], [130], 128, 1, 64, 16, True),             # group of 128 heads: one token per tile
+]
+
+
+@pytest.mark.parametrize("case", SWEEP, ids=lambda c: f"q{sum(c[0])}_h{c[2]}_{c[3]}_d{c[4]}_p{c[5]}_c{int(c[6])}")
+def test_prefill_sweep(case):
+    qo, kv, hq, hk, d, ps, causal = case
+    p = W.make_problem("sweep", qo, kv, num_qo_heads=hq, num_kv_heads=hk, head_dim=d, page_size=ps,
+                       causal=causal, seed=zlib.crc32(str(case).encode()) % 10000, pool_pages=None)
+    o, lse, _ = gpu_run(p)
+    assert_parity(o, lse, *oracle_run(p), what=str(case))
+
+
+@pytest.mark.parametrize("chunk", [128, 384])
+def test_prefill_split_kv_matches(chunk):
+    p = W.make_problem("split", [300, 40], [900, 700], num_qo_heads=8, num_kv_heads=2, head_dim=128,
+                       page_size=16, causal=True, seed=77)
+    o, lse, pl = gpu_run(p, kv_chunk=chunk)
+    assert pl.num_merges > 0
+    assert_parity(o, lse, *oracle_run(p), what=f"split {chunk}")
+
+
+def test_output_guard_regions():
+    """Writes stay inside o / lse: guard rows before and after are untouched."""
+    p = W.make_problem("guard", [33, 100], [33, 100], num_qo_heads=4, num_kv_heads=1, head_dim=64,
+                       page_size=16, causal=True, seed=5)
+    d = to_dev(p)
+    pl = pkv.plan(p.qo_indptr, p.kv_indptr, d["kv_indices"], p.kv_last_page_len, 4, 1, 64, 16, True, p.sm_scale,
+                  kv_chunk=128)
+    tq, g = p.total_q, 7
+    o_buf = torch.full((tq + 2 * g, 4, 64), 123.0, dtype=torch.bfloat16, device="cuda")
+    l_buf = torch.full((tq + 2 * g, 4), 77.0, dtype=torch.float32, device="cuda")
+    pkv.run(pl, d["q"], d["k_cache"], d["v_cache"], o=o_buf[g:g + tq], lse=l_buf[g:g + tq])
+    torch.cuda.synchronize()
+    assert torch.all(o_buf[:g] == 123.0) and torch.all(o_buf[g + tq:] == 123.0)
+    assert torch.all(l_buf[:g] == 77.0) and torch.all(l_buf[g + tq:] == 77.0)
+    assert_parity(o_buf[g:g + tq], l_buf[g:g + tq], *oracle_run(p), what="guard")
+
+
+def test_pool_permutation_bitwise_on_gpu():
+    """The physical page order does not change the GPU result at all."""
+    p = W.make_problem("perm", [150, 260], [150, 260], num_qo_heads=8, num_kv_heads=2, head_dim=128,
+                       page_size=1, causal=True, seed=9)
+    o1, l1, _ = gpu_run(p)
+    n = p.k_cache.shape[0]
+    perm = torch.randperm(n, generator=torch.Generator().manual_seed(3))
+    p2 = W.PagedProblem(**{**p.__dict__})
+    p2.k_cache = torch.empty_like(p.k_cache)
+    p2.v_cache = torch.empty_like(p.v_cache)
+    p2.k_cache[perm] = p.k_cache
+    p2.v_cache[perm] = p.v_cache
+    p2.kv_indices = perm.numpy()[p.kv_indices].astype(np.int32)
+    o2, l2, _ = gpu_run(p2)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.slow
+def test_gqa_prefill_full_size_sampled():
+    """h16/kv1/d128/ps64 at full size, in the launch configuration the bench times;
+    checked on sampled rows (first, last, page-boundary and random tokens)."""
+    p = W.gqa_prefill()
+    o, lse, _ = gpu_run(p)
+    rng = np.random.default_rng(0)
+    for b in range(p.batch):
+        L = int(p.qo_lens[b])
+        pos = sorted({0, 1, 63, 64, L // 2, L - 2, L - 1, *rng.integers(0, L, 3).tolist()})
+        o_r, l_r = oracle.paged_attention_rows(p.q, p.k_cache, p.v_cache, p.qo_indptr, p.kv_indptr,
+                                               p.kv_indices, p.kv_last_page_len, p.page_size, True,
+                                               p.sm_scale, b, pos)
+        rows = [int(p.qo_indptr[b]) + x for x in pos]
+        assert_parity(o[rows], lse[rows], o_r, l_r, what=f"req {b}")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("bl", [(16, 2048), (1, 8192)])
+def test_sparse_vs_dense_sampled(bl):
+    B, L = bl
+    sp = W.sparse_vs_dense(B, L, contiguous=False)
+    o, lse, _ = gpu_run(sp)
+    rng = np.random.default_rng(1)
+    for b in rng.choice(B, size=min(B, 2), replace=False).tolist():
+        pos = sorted({0, L - 1, *rng.integers(0, L, 4).tolist()})
+        o_r, l_r = oracle.paged_attention_rows(sp.q, sp.k_cache, sp.v_cache, sp.qo_indptr, sp.kv_indptr,
+                                               sp.kv_indices, sp.kv_last_page_len, 1, True, sp.sm_scale, b, pos)
+        rows = [int(sp.qo_indptr[b]) + x for x in pos]
+        assert_parity(o[rows], lse[rows], o_r, l_r, what=f"sparse {bl} req {b}")
+    # the dense (contiguous) layout of the same draw gives the same result
+    de = W.sparse_vs_dense(B, L, contiguous=True)
+    k = torch.empty_like(de.k_cache)
+    v = torch.empty_like(de.v_cache)
+    idx_s = torch.from_numpy(sp.kv_indices.astype(np.int64))
+    k[:len(idx_s)] = sp.k_cache[idx_s]
+    v[:len(idx_s)] = sp.v_cache[idx_s]
+    de.k_cache, de.v_cache, de.q = k, v, sp.q
+    o2, l2, _ = gpu_run(de)
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
+
+
+# --------------------------------------------------------------------------- decode
+
+DECODE_SWEEP = [
+    # kv_lens, hq, hk, d, page
+    ([1, 63, 64, 65, 3000], 32, 8, 128, 16),
+    ([500, 1], 16, 1, 128, 64),
+    ([129, 700], 8, 8, 64, 1),
+    ([2000, 333, 4], 64, 4, 128, 2),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_SWEEP, ids=lambda c: f"h{c[1]}_{c[2]}_d{c[3]}_p{c[4]}")
+@pytest.mark.parametrize("split", [False, True])
+def test_decode_sweep(case, split):
+    kv, hq, hk, d, ps = case
+    p = W.make_problem("dec", [1] * len(kv), kv, num_qo_heads=hq, num_kv_heads=hk, head_dim=d, page_size=ps,
+                       causal=False, seed=sum(kv) % 997)
+    o, lse, pl = gpu_run(p, **({"kv_chunk": 128} if split else {"disable_split_kv": True}))
+    assert pl.kind == pkv.KIND_DECODE
+    if split and max(kv) > 128:
+        assert pl.num_merges > 0
+    assert_parity(o, lse, *oracle_run(p), what=f"decode {case}")
+
+
+@pytest.mark.slow
+def test_decode_full_size():
+    """b128/h32/kv8/d128/ps16, kv_len 1024..8192, default split-KV plan: every row."""
+    p = W.paged_decode()
+    o, lse, pl = gpu_run(p)
+    assert pl.kind == pkv.KIND_DECODE
+    assert_parity(o, lse, *oracle_run(p), what="decode full")
+
+
+# --------------------------------------------------------------------------- merge
+
+def test_merge_state_kernels():
+    g = torch.Generator().manual_seed(0)
+    rows, dim = 300, 96
+    oa = torch.randn(rows, dim, generator=g)
+    ob = torch.randn(rows, dim, generator=g)
+    la = torch.randn(rows, generator=g) * 4
+    lb = torch.randn(rows, generator=g) * 4
+    la[0] = -math.inf
+    la[1] = lb[1] = -math.inf
+    o, l = pkv.merge_state(oa.cuda(), la.cuda(), ob.cuda(), lb.cuda())
+    o_ref, l_ref = oracle.merge_state(oa.numpy(), la.numpy(), ob.numpy(), lb.numpy())
+    np.testing.assert_allclose(o.cpu().double().numpy(), o_ref, rtol=1e-5, atol=1e-5)
+    assert np.array_equal(np.isneginf(l.cpu().numpy()), np.isneginf(l_ref))
+    fin = np.isfinite(l_ref)
+    np.testing.assert_allclose(l.cpu().double().numpy()[fin], l_ref[fin], atol=1e-5)
+    # n-way merge to bf16
+    n = 5
+    parts = torch.randn(n, rows, dim, generator=g)
+    lses = torch.randn(n, rows, generator=g) * 3
+    lses[:, 7] = -math.inf
+    ob16, l16 = pkv.merge_states(parts.cuda(), lses.cuda())
+    o_ref, l_ref = oracle.merge_states(list(parts.numpy()), list(lses.numpy()))
+    assert_parity(ob16, l16, o_ref, l_ref, what="merge_states")
