@@ -1,0 +1,498 @@
+"""Benchmark of the paged-KV attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--sweep]
+
+One step = one pass of the hot path over its synthetic batches: the causal
+GQA paged prefill (h16/kv1/d128/ps64, batch 8, lengths U[512, 4096]) and the
+split-KV paged decode (b128/h32/kv8/d128/ps16, kv_len U[1024, 8192]), each
+through pkv_run after an L2 flush, plus the absorbed-MLA prefill once its
+kernel is built. `value` is the prefill's causal TFLOP/s (only visible
+query/key pairs count); the decode's HBM GB/s (algorithmic bytes: K, V, Q, O,
+LSE and page indices) rides along under "decode". Kernel times come from CUDA
+events on the launching stream. `e2e` times the same prefill through the
+public API from pinned host buffers: plan + upload, H2D of q / caches / page
+table, run, D2H of O and LSE.
+
+Multi-GPU (torchrun): requests are independent, so every rank runs its own
+batch (weak scaling, no collective on the data path); the timed region is
+bracketed by barriers and the max over ranks is reported.
+
+--impl reference times the float64 CPU oracle (the only reference that exists
+for this path) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import paged_kv_attention_38_b200 as pkv  # noqa: E402
+from paged_kv_attention_38_b200 import workloads as W  # noqa: E402
+
+METRIC = "causal paged-prefill TFLOP/s & % BF16 tensor peak; decode HBM GB/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ----------------------------------------------------------------- accounting
+
+def causal_pairs(p: W.PagedProblem) -> int:
+    """Visible (query, key) pairs: bottom-right causal, or all pairs."""
+    total = 0
+    for a, b in zip(p.qo_lens.tolist(), p.kv_lens.tolist()):
+        if p.causal:
+            d = b - a
+            vis = np.clip(np.arange(a) + d + 1, 0, b)
+            total += int(vis.sum())
+        else:
+            total += a * b
+    return total
+
+
+def attention_flops(p: W.PagedProblem) -> float:
+    """2 FLOPs per multiply-add for Q.K^T (width head_dim [+ rope]) and P.V, per visible pair and head."""
+    return 2.0 * (p.head_dim + p.head_dim_pe + p.head_dim_v) * p.num_qo_heads * causal_pairs(p)
+
+
+def decode_bytes(p: W.PagedProblem) -> float:
+    """Algorithmic HBM bytes of a decode pass: K and V rows of every request once,
+    Q and O (bf16), LSE (fp32) and the page indices."""
+    kv = 2 * 2 * p.num_kv_heads * p.head_dim * int(p.kv_lens.sum())
+    q = 2 * p.total_q * p.num_qo_heads * p.head_dim
+    o = 2 * p.total_q * p.num_qo_heads * p.head_dim_v
+    lse = 4 * p.total_q * p.num_qo_heads
+    idx = 4 * len(p.kv_indices)
+    return float(kv + q + o + lse + idx)
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- our arm
+
+class Case:
+    """A problem resident in HBM with its plan, ready to run."""
+
+    def __init__(self, p: W.PagedProblem, device, **plan_kw):
+        self.p = p
+        self.idx = torch.from_numpy(p.kv_indices.astype(np.int32)).to(device)
+        if p.is_mla:
+            self.q_nope, self.q_pe = p.q_nope.to(device), p.q_pe.to(device)
+            self.ckv, self.kpe = p.ckv_cache.to(device), p.kpe_cache.to(device)
+            self.plan = pkv.plan_mla(p.qo_indptr, p.kv_indptr, self.idx, p.kv_last_page_len, p.num_qo_heads,
+                                     p.head_dim, p.head_dim_pe, p.page_size, p.causal, p.sm_scale, **plan_kw)
+            self.o = torch.empty(p.total_q, p.num_qo_heads, p.head_dim_v, dtype=torch.bfloat16, device=device)
+        else:
+            self.q, self.k, self.v = p.q.to(device), p.k_cache.to(device), p.v_cache.to(device)
+            self.plan = pkv.plan(p.qo_indptr, p.kv_indptr, self.idx, p.kv_last_page_len, p.num_qo_heads,
+                                 p.num_kv_heads, p.head_dim, p.page_size, p.causal, p.sm_scale, **plan_kw)
+            self.o = torch.empty(p.total_q, p.num_qo_heads, p.head_dim_v, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(p.total_q, p.num_qo_heads, dtype=torch.float32, device=device)
+
+    @property
+    def launches(self) -> int:
+        return 1 + (1 if self.plan.num_merges > 0 else 0)
+
+    def run(self):
+        if self.p.is_mla:
+            pkv.run_mla(self.plan, self.q_nope, self.q_pe, self.ckv, self.kpe, self.o, self.lse)
+        else:
+            pkv.run(self.plan, self.q, self.k, self.v, self.o, self.lse)
+
+
+def time_case(case: Case, flush: torch.Tensor, steps: int, warmup: int):
+    """Median and mean kernel time (ms) of `case.run`, L2 flushed before every launch."""
+    for _ in range(warmup):
+        flush.zero_()
+        case.run()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        case.run()
+        b.record()
+        times.append((a, b))
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in times]
+    return float(np.median(ms)), float(np.mean(ms))
+
+
+def e2e_prefill(p: W.PagedProblem, device, steps: int, warmup: int):
+    """Prefill through the public API from pinned host buffers, copies inside the timed region."""
+    hq = p.q.pin_memory()
+    hk = p.k_cache.pin_memory()
+    hv = p.v_cache.pin_memory()
+    hidx = torch.from_numpy(p.kv_indices.astype(np.int32)).pin_memory()
+    ho = torch.empty(p.total_q, p.num_qo_heads, p.head_dim_v, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty(p.total_q, p.num_qo_heads, dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(hq, device=device), torch.empty_like(hk, device=device), torch.empty_like(hv, device=device)
+    didx = torch.empty_like(hidx, device=device)
+    do = torch.empty_like(ho, device=device)
+    dl = torch.empty_like(hl, device=device)
+    plans = []
+
+    def step():
+        didx.copy_(hidx, non_blocking=True)
+        pl = pkv.plan(p.qo_indptr, p.kv_indptr, didx, p.kv_last_page_len, p.num_qo_heads, p.num_kv_heads,
+                      p.head_dim, p.page_size, p.causal, p.sm_scale)
+        plans.append(pl)  # keep the plan (and its pinned staging) alive until the stream drains
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        pkv.run(pl, dq, dk, dv, do, dl)
+        ho.copy_(do, non_blocking=True)
+        hl.copy_(dl, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    plans.clear()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + hidx.numel() * 4
+    d2h = ho.numel() * 2 + hl.numel() * 4
+    return ms, h2d, d2h
+
+
+def cpu_baseline(seconds_target: float = 15.0):
+    """The float64 oracle, as it stands, on a bounded sample of the prefill workload:
+    whole requests of the h16/kv1/d128/ps64 batch, shortest first, until the target
+    CPU time is spent. Returns TFLOP/s on the sample's causal FLOPs."""
+    import oracle
+    p = W.gqa_prefill()
+    order = np.argsort(p.qo_lens)
+    t0 = time.perf_counter()
+    flops, done = 0.0, []
+    for b in order.tolist():
+        oracle.paged_attention(p.q, p.k_cache, p.v_cache, p.qo_indptr, p.kv_indptr, p.kv_indices,
+                               p.kv_last_page_len, p.page_size, True, p.sm_scale, requests=[b])
+        L = int(p.qo_lens[b])
+        flops += 2.0 * (2 * p.head_dim) * p.num_qo_heads * L * (L + 1) / 2
+        done.append((b, L))
+        if time.perf_counter() - t0 > seconds_target:
+            break
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(done)} of 8 requests of the h16/kv1/d128/ps64 prefill batch "
+                      f"(qo_len {[l for _, l in done]}), float64 NumPy, {dt:.1f} s"}
+
+
+def dist_setup(n_gpus: int):
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def run_ours(args):
+    rank, world, local = dist_setup(args.gpus)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks, peak_kind = load_peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    if args.only:
+        return run_only(args, device, flush)
+    pre = Case(W.gqa_prefill(), device)
+    dec = Case(W.paged_decode(), device)
+    cases = [pre, dec]
+    mla = None
+    try:
+        mla = Case(W.mla_prefill(), device)
+        mla.run()
+        torch.cuda.synchronize()
+        cases.append(mla)
+    except pkv.PkvError:
+        mla = None
+
+    # warm-up steps
+    for _ in range(args.warmup):
+        for c in cases:
+            flush.zero_()
+            c.run()
+    barrier(world)
+
+    ev = {id(c): [] for c in cases}
+    sampler = ClockSampler(local)
+    with sampler:
+        barrier(world)
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record()
+        for _ in range(args.steps):
+            for c in cases:
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                c.run()
+                b.record()
+                ev[id(c)].append((a, b))
+        t_end.record()
+        barrier(world)
+    clocks = sampler.summary()
+
+    def mean_ms(c):
+        return float(np.mean([a.elapsed_time(b) for a, b in ev[id(c)]]))
+
+    pre_ms = max_over_ranks(mean_ms(pre), world)
+    dec_ms = max_over_ranks(mean_ms(dec), world)
+    mla_ms = max_over_ranks(mean_ms(mla), world) if mla else None
+    step_ms = pre_ms + dec_ms + (mla_ms or 0.0)
+
+    pre_flops = attention_flops(pre.p)
+    dec_bytes = decode_bytes(dec.p)
+    tflops = pre_flops * world / (pre_ms * 1e-3) / 1e12
+    per_gpu_tflops = pre_flops / (pre_ms * 1e-3) / 1e12
+    dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
+
+    # e2e through the public API with host buffers
+    e2e_ms, h2d, d2h = e2e_prefill(pre.p, device, max(2, min(args.steps, 10)), 2)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+
+    peak_burst = float(peaks["bf16_tflops"])
+    peak_sust = float(peaks.get("bf16_tflops_sustained", peak_burst))
+    hbm = float(peaks["hbm_gbs"])
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            tj = json.load(f)
+        if tj.get("kernel_version") == pkv.load_library().pkv_version().decode():
+            traffic = tj.get("prefill_bytes_per_launch")
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded bf16 N(0,1), random page permutation)",
+        "config": {
+            "workload": "gqa_paged_prefill_causal_h16_kv1_d128_ps64: batch 8, qo_len=kv_len U[512,4096], "
+                        "page_size 64, permuted pool",
+            "lengths": pre.p.qo_lens.tolist(),
+            "parallelism": f"dp{world} (independent batches per GPU)",
+            "l2": "flushed (256 MiB write) before every timed launch",
+            "step": "prefill h16/kv1/d128/ps64 + decode b128/h32/kv8/d128/ps16" + (" + MLA h16/ckv512/kpe64/ps1" if mla else ""),
+        },
+        "pct_bf16_peak": round(100 * per_gpu_tflops / peak_burst, 2),
+        "prefill": {"ms": round(pre_ms, 4), "flops": pre_flops, "tflops_per_gpu": round(per_gpu_tflops, 2),
+                    "units": pre.plan.num_units, "merges": pre.plan.num_merges},
+        "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "ms": round(dec_ms, 4), "bytes": dec_bytes,
+                   "frac": round(dec_gbs / hbm, 4), "peak": hbm, "peak_kind": peak_kind,
+                   "units": dec.plan.num_units, "merges": dec.plan.num_merges,
+                   "workload": "paged_decode_b128_h32_kv8_d128_ps16, kv_len U[1024,8192]"},
+        "roofline": {"bound": "tensor", "achieved": round(per_gpu_tflops, 2), "peak": peak_burst,
+                     "unit": "TFLOP/s", "frac": round(per_gpu_tflops / peak_burst, 4),
+                     "frac_of_sustained": round(per_gpu_tflops / peak_sust, 4),
+                     "peak_kind": f"{peak_kind} burst bf16 (kernel timed alone between L2 flushes)",
+                     "traffic": traffic, "kernel": "prefill_kernel<128>"},
+        "e2e": {"value": round(pre_flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "includes": "plan + upload + H2D(q, k, v, kv_indices) + run + D2H(o, lse)"},
+        "gpu_launches": int(args.steps * sum(c.launches for c in cases)),
+        "clocks": clocks,
+    }
+    if mla:
+        mla_flops = attention_flops(mla.p)
+        line["mla"] = {"value": round(mla_flops / (mla_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                       "ms": round(mla_ms, 4), "flops": mla_flops,
+                       "workload": "mla_paged_prefill_causal_h16_ckv512_kpe64_ps1, batch 4, U[256,2048]"}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if args.sweep:
+        line["sparse_vs_dense"] = sparse_dense_sweep(device, flush, args)
+    print(json.dumps(line), flush=True)
+
+
+def run_only(args, device, flush):
+    """One workload alone (for profiler captures): W warm-up and K timed launches."""
+    makers = {"prefill": W.gqa_prefill, "decode": W.paged_decode, "mla": W.mla_prefill,
+              "sparse": lambda: W.sparse_vs_dense(16, 2048, False),
+              "dense": lambda: W.sparse_vs_dense(16, 2048, True)}
+    c = Case(makers[args.only](), device)
+    med, mean = time_case(c, flush, args.steps, args.warmup)
+    f = attention_flops(c.p)
+    print(json.dumps({"only": args.only, "ms_median": med, "ms_mean": mean,
+                      "tflops": f / (med * 1e-3) / 1e12,
+                      "gbs": decode_bytes(c.p) / (med * 1e-3) / 1e9 if args.only == "decode" else None,
+                      "units": c.plan.num_units, "merges": c.plan.num_merges}), flush=True)
+
+
+def sparse_dense_sweep(device, flush, args):
+    """Vector-sparse (page_size 1, scattered slots) vs contiguous ragged KV, same problem."""
+    out = []
+    for B, L in W.SPARSE_DENSE_SWEEP:
+        sp = W.sparse_vs_dense(B, L, contiguous=False)
+        cs = Case(sp, device)
+        de = W.sparse_vs_dense(B, L, contiguous=True)
+        cd = Case(de, device)
+        ms_s, _ = time_case(cs, flush, max(5, args.steps), 3)
+        ms_d, _ = time_case(cd, flush, max(5, args.steps), 3)
+        f = attention_flops(sp)
+        out.append({"B": B, "L": L, "sparse_tflops": round(f / ms_s / 1e9, 1),
+                    "dense_tflops": round(f / ms_d / 1e9, 1), "ratio": round(ms_d / ms_s, 3)})
+        del cs, cd
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", 0))
+    if rank != 0:
+        return
+    import oracle
+    p = W.gqa_prefill()
+    b = int(np.argmin(p.qo_lens))
+    L = int(p.qo_lens[b])
+    flops = 2.0 * (2 * p.head_dim) * p.num_qo_heads * L * (L + 1) / 2
+    for _ in range(args.warmup):
+        pass  # the oracle has no state to warm; warm-up steps are not repeated on the CPU
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.paged_attention(p.q, p.k_cache, p.v_cache, p.qo_indptr, p.kv_indptr, p.kv_indices,
+                               p.kv_last_page_len, p.page_size, True, p.sm_scale, requests=[b])
+    dt = (time.perf_counter() - t0) / args.steps
+    value = flops / dt / 1e12
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"request {b} (qo_len = kv_len = {L}) of the h16/kv1/d128/ps64 prefill batch per step, "
+              f"float64 NumPy oracle")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "gqa_paged_prefill_causal_h16_kv1_d128_ps64 (one request per step)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--sweep", action="store_true", help="also run the vector-sparse vs dense sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "decode", "mla", "sparse", "dense"], default=None,
+                    help="time one workload alone (profiler captures)")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -13,7 +13,7 @@
 
 namespace pkv {
 cudaError_t launch_prefill(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
-                           const void*, void*, float*, cudaStream_t);
+                           const void*, int32_t, void*, float*, cudaStream_t);
 cudaError_t launch_decode(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
                           const void*, void*, float*, cudaStream_t);
 cudaError_t launch_mla(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
@@ -193,7 +193,7 @@ pkv_status pkv_run(const pkv_plan* p, const void* q, const void* k_cache, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = s.kind == kKindDecode
                       ? launch_decode(s.geom, p->dv, p->kv_indices, q, k_cache, v_cache, o, lse, st)
-                      : launch_prefill(s.geom, p->dv, p->kv_indices, q, k_cache, v_cache, o, lse, st);
+                      : launch_prefill(s.geom, p->dv, p->kv_indices, q, k_cache, v_cache, num_pages, o, lse, st);
   if (e == cudaSuccess) e = launch_merge_tasks(s.geom, p->dv, o, lse, st);
   if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
   return PKV_OK;

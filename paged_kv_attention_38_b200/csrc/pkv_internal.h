@@ -7,7 +7,8 @@
 
 namespace pkv {
 
-constexpr int kBlockM = 128;   // packed (token, head-in-group) rows per prefill tile
+constexpr int kBlockM = 128;   // packed (token, head-in-group) rows per tensor-core tile (TMEM lanes)
+constexpr int kPrefillUnitRows = 256;  // packed rows per prefill work unit (two tiles share K/V)
 constexpr int kBlockN = 128;   // KV slots per prefill KV tile
 constexpr int kDecodeRows = 16;  // packed rows per decode unit (mma.sync M)
 constexpr int kDecodeTileN = 64;  // KV slots per decode pipeline stage
@@ -68,6 +69,7 @@ struct LaunchGeom {
   int32_t part_rows;      // rows per partial slot
   int32_t num_units;
   int32_t num_merge;
+  int32_t total_q;        // rows of q (tokens)
 };
 
 // Device pointers into the workspace after upload.

@@ -88,10 +88,12 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
 
   const int32_t num_sms = in.num_sms > 0 ? in.num_sms : 148;
   s.num_sms = num_sms;
-  const int32_t tile_rows = s.kind == kKindDecode ? kDecodeRows : kBlockM;
-  // MLA tiles pack tokens x heads the same way, with a single latent "kv head".
-  const int32_t mla_tile_rows = kBlockM;
-  const int32_t rows_per_tile = s.kind == kKindMla ? mla_tile_rows : tile_rows;
+  // Rows per work unit: decode packs one token's group of heads into an mma.sync
+  // tile; prefill units hold two 128-row tensor-core tiles that share K/V; MLA
+  // packs tokens x heads the same way with one latent "kv head".
+  const int32_t rows_per_tile = s.kind == kKindDecode ? kDecodeRows
+                                : s.kind == kKindMla  ? kBlockM
+                                                      : kPrefillUnitRows;
 
   // ---- tiles
   std::vector<Tile> tiles;
@@ -172,6 +174,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   gm.part_rows = rows_per_tile;
   gm.num_units = (int32_t)s.units.size();
   gm.num_merge = (int32_t)s.merges.size();
+  gm.total_q = in.batch > 0 ? in.qo_indptr[in.batch] : 0;
   *out = std::move(s);
   return 0;
 }

@@ -3,27 +3,40 @@
 // What it computes (flashinfer-trace discussion #15, definition
 // gqa_paged_prefill_causal_h16_kv1_d128_ps64 and "Notes on fa3_gqa_prefill_v1";
 // FlashInfer 0.2 release, "FlashAttention-3 template with block/vector
-// sparsity"): for each work unit (request, kv head, 128 packed query rows,
+// sparsity"): for each work unit (request, kv head, 256 packed query rows,
 // KV range), O = softmax(sm_scale Q K^T + causal mask) V over the keys the
-// page table lists, plus the base-2 LSE of every row. The K/V rows of a tile
-// are gathered page by page through kv_indices, so page_size = 1 (vector
-// sparsity) and page_size = 64 run the same code; only the gather differs
-// from dense attention.
+// page table lists, plus the base-2 LSE of every row. K/V rows are gathered
+// page by page through kv_indices: whole pages by TMA when page_size >= 8,
+// single rows by 16-byte cp.async for page_size 1..4 (vector sparsity). The
+// gather is the only difference from dense attention.
 //
-// CTA layout (288 threads, one work unit per CTA):
-//   warps 0-3  softmax + epilogue. Thread i owns query row i = TMEM lane i.
-//   warp  4    TMEM allocator and MMA issuer (one lane issues tcgen05.mma).
-//   warps 5-8  producer: cp.async gather of Q once, then K/V tiles of 128 keys
-//              into a 2-stage ring, 16-byte copies, 128-byte swizzled rows.
-// TMEM (512 columns): S double buffer at columns [0,128) and [128,256), O at
-// [256, 256 + D). P goes through shared memory as the A operand of P.V.
+// CTA layout (384 threads, one work unit of two 128-row query tiles):
+//   warps 0-3  softmax of query tile 0 (thread i owns row i = TMEM lane i)
+//   warps 4-7  softmax of query tile 1
+//   warp  8    TMEM allocator + MMA issuer (one lane)
+//   warps 9-11 producer: TMA (one lane) or cp.async gather (96 threads)
+// Shared memory: Q tiles (2 x 128 x D) and a 4-slot ring of 128 x D K or V
+// tiles, all in 128-byte swizzled rows. TMEM (512 columns): S0 [0,128),
+// S1 [128,256), O0 [256,384), O1 [384,512). After softmax reads S_i it writes
+// P_i (bf16, two per column) over the first 64 columns of S_i, and the P.V
+// MMA takes P_i straight from TMEM as its A operand.
 //
-// Per KV tile j the MMA warp issues S_j = Q K_j^T (into S buffer j%2) before
-// O += P_{j-1} V_{j-1}, so the softmax of tile j overlaps the P.V of tile j-1.
-// Online softmax runs in the base-2 domain: s' = s * sm_scale * log2(e),
-// p = 2^(s' - m); O is rescaled in TMEM only when a row's max grows.
+// Per KV tile j the MMA warp issues, in order:
+//   O0 += P0 V_j,  S0 = Q0 K_{j+1}^T,  O1 += P1 V_j,  S1 = Q1 K_{j+1}^T
+// so the softmax of one query tile overlaps the MMAs of the other. The tensor
+// core executes a CTA's MMAs in issue order, so S_i(j+1) overwrites P_i(j)
+// only after O_i += P_i(j) V_j has read it, and the commit that signals S_i(j+1)
+// also covers O_i += P_i(j) V_j: when softmax sees S_i(j+1), O_i is stable and
+// may be rescaled in place.
+//
+// Online softmax runs in the base-2 domain (s' = s * sm_scale * log2 e,
+// p = 2^(s' - m)). A row's running max m is only moved when the new tile's
+// max exceeds it by more than 8 (p then stays below 2^8 in fp32 / bf16), so O
+// is rescaled in TMEM a few times per row instead of once per tile.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "pkv_internal.h"
 #include "sm100_ptx.cuh"
@@ -32,40 +45,43 @@ namespace pkv {
 
 namespace {
 
-constexpr int kThreads = 288;
-constexpr int kSoftmaxThreads = 128;
-constexpr int kProducerThreads = 128;
-constexpr int kProducerWarp0 = 5;
-constexpr int kMmaWarp = 4;
-constexpr int kStages = 2;
+constexpr int kTileM = 128;
+constexpr int kTiles = 2;
+constexpr int kSlots = 4;
+constexpr int kThreads = 384;
+constexpr int kMmaWarp = 8;
+constexpr int kProdWarp0 = 9;
+constexpr int kProdThreads = 96;
 constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;
+static_assert(kTileM * kTiles == kPrefillUnitRows, "unit rows");
 
-// Byte offset of 16-byte chunk `ch` (of row length D/8 chunks) of row `r` in a
-// [128 x D] bf16 tile stored as D/64 column blocks of [128 rows x 128 B] with
-// the 128-byte swizzle (chunk index XOR row % 8).
+// Byte offset of 16-byte chunk `ch` of row `r` in a [128 x D] bf16 tile held as
+// D/64 column blocks of [128 rows x 128 B], 128-byte swizzle (chunk ^ row % 8):
+// the layout TMA SWIZZLE_128B writes and the UMMA SW128 descriptors read.
 __device__ __forceinline__ uint32_t tile_off(int r, int ch) {
-  return (uint32_t)((ch >> 3) * (kBlockM * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+  return (uint32_t)((ch >> 3) * (kTileM * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
 }
 
 template <int D>
 struct __align__(1024) Smem {
-  __nv_bfloat16 q[kBlockM * D];
-  __nv_bfloat16 k[kStages][kBlockN * D];
-  __nv_bfloat16 v[kStages][kBlockN * D];
-  __nv_bfloat16 p[kBlockM * kBlockN];
+  __nv_bfloat16 q[kTiles][kTileM * D];
+  __nv_bfloat16 kv[kSlots][kBlockN * D];
   uint64_t q_full;
-  uint64_t k_full[kStages];
-  uint64_t v_full[kStages];
-  uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t s_free[2];
-  uint64_t p_full;
-  uint64_t o_done;
+  uint64_t full[kSlots];
+  uint64_t empty[kSlots];
+  uint64_t s_full[kTiles];
+  uint64_t p_full[kTiles];
+  uint64_t o_final;
+  int32_t rowsrc[kBlockN];  // cp.async gather: pool row of each tile row, -1 = zero fill
   uint32_t tmem_base;
   int abort_flag;
 };
 
 struct Args {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
@@ -74,6 +90,9 @@ struct Args {
   float* lse;
   LaunchGeom g;
   DeviceView dv;
+  int32_t q_tma;      // Q tiles by TMA (group divides 128) or by cp.async
+  int32_t kv_tma;     // K/V pages by TMA (page_size >= 8) or by cp.async rows
+  int32_t oob_row;    // a pool row index past the end: TMA zero-fills it
 };
 
 template <int D>
@@ -90,18 +109,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   const int n_tiles = (unit.kv_hi - unit.kv_lo + kBlockN - 1) / kBlockN;
 
   if (tid == 0) {
-    mbar_init(&sm.q_full, kProducerThreads);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.k_full[s], kProducerThreads);
-      mbar_init(&sm.v_full[s], kProducerThreads);
-      mbar_init(&sm.kv_empty[s], 1);
+    mbar_init(&sm.q_full, a.q_tma ? 1 : kProdThreads);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&sm.full[s], a.kv_tma ? 1 : kProdThreads);
+      mbar_init(&sm.empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_free[s], kSoftmaxThreads);
+    for (int i = 0; i < kTiles; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], kTileM);
     }
-    mbar_init(&sm.p_full, kSoftmaxThreads);
-    mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.o_final, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -115,234 +132,292 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   const uint32_t tmem = sm.tmem_base;
   WaitCtx wc{&sm.abort_flag, a.dv.status};
 
-  if (warp >= kProducerWarp0) {
-    // ------------------------------------------------------------ producer
-    const int pt = tid - kProducerWarp0 * 32;
-    constexpr int kChunks = D / 8;  // 16-byte chunks per row
-    const size_t head_stride_q = (size_t)a.g.num_qo_heads * D;
-    // Q tile: packed row r -> token q_start + (row0 + r) / G, head kv_head*G + (row0 + r) % G
-    for (int c = pt; c < kBlockM * kChunks; c += kProducerThreads) {
-      const int r = c / kChunks, ch = c % kChunks;
-      const bool ok = r < unit.rows;
-      const __nv_bfloat16* src = a.q;
-      if (ok) {
-        const int pr = unit.row0 + r;
-        const int t = req.q_start + pr / G;
-        const int h = unit.kv_head * G + pr % G;
-        src = a.q + (size_t)t * head_stride_q + (size_t)h * D + ch * 8;
-      }
-      cp_async_16(smem_u32(sm.q) + tile_off(r, ch), src, ok ? 16u : 0u);
-    }
-    cp_async_commit();
+  if (warp >= kProdWarp0) {
+    // ================================================================ producer
+    const int pt = tid - kProdWarp0 * 32;
+    constexpr int kChunks = D / 8;
     const int P = a.g.page_size, shift = a.g.page_shift, Hk = a.g.num_kv_heads;
-    auto load_kv = [&](const __nv_bfloat16* base, __nv_bfloat16* dst, int j) {
-      for (int c = pt; c < kBlockN * kChunks; c += kProducerThreads) {
-        const int r = c / kChunks, ch = c % kChunks;
-        const int pos = unit.kv_lo + j * kBlockN + r;
-        const bool ok = pos < unit.kv_hi;
-        const __nv_bfloat16* src = base;
-        if (ok) {
-          const int page = __ldg(a.kv_indices + req.page0 + (pos >> shift));
-          const int slot = pos & (P - 1);
-          src = base + (((size_t)page * P + slot) * Hk + unit.kv_head) * D + ch * 8;
-        }
-        cp_async_16(smem_u32(dst) + tile_off(r, ch), src, ok ? 16u : 0u);
+    if (pt == 0) {
+      if (a.q_tma) tma_prefetch_desc(&a.tm_q);
+      if (a.kv_tma) {
+        tma_prefetch_desc(&a.tm_k);
+        tma_prefetch_desc(&a.tm_v);
       }
-      cp_async_commit();
-    };
-    // Each group is signalled once the next one is in flight (wait_group 1),
-    // after this thread's fence.proxy.async makes its copies visible to the
-    // tensor core.
-    for (int j = 0; j < n_tiles; ++j) {
-      const int s = j & 1;
-      if (j >= kStages) mbar_wait(&sm.kv_empty[s], ((j >> 1) - 1) & 1, wc);
-      load_kv(a.k, sm.k[s], j);
-      cp_async_wait<1>();
-      fence_proxy_async_smem();
-      if (j == 0) mbar_arrive(&sm.q_full);
-      else mbar_arrive(&sm.v_full[(j - 1) & 1]);
-      load_kv(a.v, sm.v[s], j);
-      cp_async_wait<1>();
-      fence_proxy_async_smem();
-      mbar_arrive(&sm.k_full[s]);
+    }
+    // ---- Q tiles (nothing to load when the unit has no key: the CTA only writes zeros)
+    if (n_tiles == 0) {
+    } else if (a.q_tma) {
+      if (pt == 0) {
+        mbar_arrive_expect_tx(&sm.q_full, kTiles * kTileM * D * 2);
+        for (int i = 0; i < kTiles; ++i) {
+          const int t0 = (unit.row0 + i * kTileM) / G;
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_3d(smem_u32(sm.q[i]) + h * (kTileM * 128), &a.tm_q, &sm.q_full, h * 64, unit.kv_head * G,
+                        req.q_start + t0);
+        }
+      }
+    } else {
+      const size_t head_stride = (size_t)a.g.num_qo_heads * D;
+      for (int c = pt; c < kTiles * kTileM * kChunks; c += kProdThreads) {
+        const int r = c / kChunks, ch = c % kChunks;
+        const bool ok = r < unit.rows;
+        const __nv_bfloat16* src = a.q;
+        if (ok) {
+          const int pr = unit.row0 + r;
+          src = a.q + (size_t)(req.q_start + pr / G) * head_stride + (size_t)(unit.kv_head * G + pr % G) * D + ch * 8;
+        }
+        cp_async_16(smem_u32(sm.q[r / kTileM]) + tile_off(r % kTileM, ch), src, ok ? 16u : 0u);
+      }
+      cp_async_arrive_noinc(&sm.q_full);
+    }
+    // ---- K / V items: item 2j is K_j, item 2j+1 is V_j, slot = item % kSlots
+    const int n_pages_req = (req.kv_len + P - 1) >> shift;
+    for (int k = 0; k < 2 * n_tiles; ++k) {
+      const int slot = k & (kSlots - 1);
+      const int j = k >> 1;
+      const bool is_v = k & 1;
+      const int pos0 = unit.kv_lo + j * kBlockN;
+      if (a.kv_tma) {
+        if (pt == 0) {
+          if (k >= kSlots) mbar_wait(&sm.empty[slot], ((k >> 2) - 1) & 1, wc);
+          mbar_arrive_expect_tx(&sm.full[slot], kBlockN * D * 2);
+          const CUtensorMap* tm = is_v ? &a.tm_v : &a.tm_k;
+          const uint32_t dst = smem_u32(sm.kv[slot]);
+          if (P >= kBlockN) {
+            const int page = __ldg(a.kv_indices + req.page0 + (pos0 >> shift));
+            const int row = page * P + (pos0 & (P - 1));
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h) tma_load_3d(dst + h * (kTileM * 128), tm, &sm.full[slot], h * 64, unit.kv_head, row);
+          } else {
+            const int npc = kBlockN >> shift;
+            const int lp0 = pos0 >> shift;
+            for (int pi = 0; pi < npc; ++pi) {
+              const int lp = lp0 + pi;
+              const int row = lp < n_pages_req ? __ldg(a.kv_indices + req.page0 + lp) * P : a.oob_row;
+#pragma unroll
+              for (int h = 0; h < D / 64; ++h)
+                tma_load_3d(dst + h * (kTileM * 128) + pi * P * 128, tm, &sm.full[slot], h * 64, unit.kv_head, row);
+            }
+          }
+        }
+      } else {
+        if (k >= kSlots) mbar_wait(&sm.empty[slot], ((k >> 2) - 1) & 1, wc);
+        if (!is_v) {
+          named_bar_sync(1, kProdThreads);  // the previous tile's copies have all been issued
+          for (int r = pt; r < kBlockN; r += kProdThreads) {
+            const int pos = pos0 + r;
+            int src = -1;
+            if (pos < unit.kv_hi) src = __ldg(a.kv_indices + req.page0 + (pos >> shift)) * P + (pos & (P - 1));
+            sm.rowsrc[r] = src;
+          }
+          named_bar_sync(1, kProdThreads);
+        }
+        const __nv_bfloat16* base = is_v ? a.v : a.k;
+        const uint32_t dst = smem_u32(sm.kv[slot]);
+        for (int c = pt; c < kBlockN * kChunks; c += kProdThreads) {
+          const int r = c / kChunks, ch = c % kChunks;
+          const int src = sm.rowsrc[r];
+          const __nv_bfloat16* g = src >= 0 ? base + ((size_t)src * Hk + unit.kv_head) * D + ch * 8 : base;
+          cp_async_16(dst + tile_off(r, ch), g, src >= 0 ? 16u : 0u);
+        }
+        cp_async_arrive_noinc(&sm.full[slot]);
+      }
     }
     cp_async_wait<0>();
-    fence_proxy_async_smem();
-    if (n_tiles > 0) mbar_arrive(&sm.v_full[(n_tiles - 1) & 1]);
+    // Make sure no TMA write into this CTA's shared memory is still in flight at exit.
+    if (pt == 0 && n_tiles > 0) {
+      if (a.q_tma) mbar_drain(&sm.q_full, 0);
+      if (a.kv_tma)
+        for (int k = 2 * n_tiles - 1; k >= 0 && k >= 2 * n_tiles - kSlots; --k)
+          mbar_drain(&sm.full[k & (kSlots - 1)], (k >> 2) & 1);
+    }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+    // ================================================================ MMA issuer
     if (lane == 0 && n_tiles > 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
-      const uint32_t q_addr = smem_u32(sm.q);
-      const uint32_t p_addr = smem_u32(sm.p);
-      const uint32_t o_tmem = tmem + 256;
-      auto issue_pv = [&](int jj) {
-        const int sp = jj & 1;
-        mbar_wait(&sm.p_full, jj & 1, wc);
-        mbar_wait(&sm.v_full[sp], (jj >> 1) & 1, wc);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kTileM, kBlockN, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kTileM, D, true);
+      auto wait_item = [&](int k) {
+        mbar_wait(&sm.full[k & (kSlots - 1)], (k >> 2) & 1, wc);
+        fence_proxy_async_smem();  // cp.async rows were written through the generic proxy
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm.v[sp]);
-#pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          const uint64_t da = sdesc_sw128(p_addr + (kk >> 2) * (kBlockM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t db = sdesc_sw128(v_addr + kk * 16 * 128, kBlockN * 128, 1024);
-          umma_bf16(o_tmem, da, db, idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&sm.o_done);
-        umma_commit(&sm.kv_empty[sp]);
       };
-      mbar_wait(&sm.q_full, 0, wc);
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j & 1;
-        mbar_wait(&sm.k_full[s], (j >> 1) & 1, wc);
-        if (j >= 2) mbar_wait(&sm.s_free[s], ((j >> 1) - 1) & 1, wc);
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm.k[s]);
+      auto issue_s = [&](int i, int j) {
+        const uint32_t k_addr = smem_u32(sm.kv[(2 * j) & (kSlots - 1)]);
+        const uint32_t q_addr = smem_u32(sm.q[i]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kBlockM * 128) + (kk & 3) * 32;
-          umma_bf16(tmem + s * kBlockN, sdesc_sw128(q_addr + off, 16, 1024),
-                    sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          const uint32_t off = (kk >> 2) * (kTileM * 128) + (kk & 3) * 32;
+          umma_bf16(tmem + i * kBlockN, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
+                    idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&sm.s_full[s]);
-        if (j >= 1) issue_pv(j - 1);
+      };
+      auto issue_pv = [&](int i, int j) {
+        const uint32_t v_addr = smem_u32(sm.kv[(2 * j + 1) & (kSlots - 1)]);
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk)
+          umma_bf16_ts(tmem + 256 + i * 128, tmem + i * kBlockN + kk * 8,
+                       sdesc_sw128(v_addr + kk * 16 * 128, kBlockN * 128, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      mbar_wait(&sm.q_full, 0, wc);
+      fence_proxy_async_smem();
+      wait_item(0);
+      issue_s(0, 0);
+      umma_commit(&sm.s_full[0]);
+      issue_s(1, 0);
+      umma_commit(&sm.s_full[1]);
+      umma_commit(&sm.empty[0]);
+      for (int j = 0; j < n_tiles; ++j) {
+        const bool more = j + 1 < n_tiles;
+        mbar_wait(&sm.p_full[0], j & 1, wc);
+        wait_item(2 * j + 1);
+        issue_pv(0, j);
+        if (more) {
+          wait_item(2 * j + 2);
+          issue_s(0, j + 1);
+          umma_commit(&sm.s_full[0]);
+        }
+        mbar_wait(&sm.p_full[1], j & 1, wc);
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(&sm.empty[(2 * j + 1) & (kSlots - 1)]);
+        if (more) {
+          issue_s(1, j + 1);
+          umma_commit(&sm.s_full[1]);
+          umma_commit(&sm.empty[(2 * j + 2) & (kSlots - 1)]);
+        }
       }
-      issue_pv(n_tiles - 1);
+      umma_commit(&sm.o_final);
+      mbar_drain(&sm.o_final, 0);  // no MMA may still run when TMEM is released
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax
-    const int r = tid;  // query row == TMEM lane
-    const bool row_ok = r < unit.rows;
-    const int pr = unit.row0 + (row_ok ? r : 0);
-    const int t = pr / G;  // token index within the request
-    int limit = unit.kv_hi;  // exclusive bound on key position for this row
+    // ================================================================ softmax
+    const int ti = warp >> 2;          // query tile
+    const int r = tid & (kTileM - 1);  // row in tile == TMEM lane
+    const int ru = ti * kTileM + r;    // row in unit
+    const bool row_ok = ru < unit.rows;
+    const int pr = unit.row0 + (row_ok ? ru : 0);
+    const int t = pr / G;
+    int limit = unit.kv_hi;
     if (a.g.causal) limit = min(limit, t + req.kv_len - req.qo_len + 1);
     const float scale = a.g.sm_scale_log2;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    const uint32_t o_tmem = lane_base + 256;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t s_tm = lane_base + ti * kBlockN;
+    const uint32_t o_tm = lane_base + 256 + ti * 128;
     float m = -INFINITY, l = 0.f;
-    const uint32_t p_addr = smem_u32(sm.p);
-    float sv[kBlockN];
     for (int j = 0; j < n_tiles; ++j) {
-      const int s = j & 1;
-      mbar_wait(&sm.s_full[s], (j >> 1) & 1, wc);
+      mbar_wait(&sm.s_full[ti], j & 1, wc);
       tc_fence_after();
+      float sv[kBlockN];
 #pragma unroll
-      for (int c = 0; c < kBlockN; c += 32) tmem_ld32(lane_base + s * kBlockN + c, sv + c);
+      for (int c = 0; c < kBlockN; c += 32) tmem_ld32(s_tm + c, sv + c);
       tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&sm.s_free[s]);
       const int kv0 = unit.kv_lo + j * kBlockN;
+      const bool whole = kv0 + kBlockN <= limit;
       float mx = -INFINITY;
-      if (kv0 + kBlockN <= limit) {
+      if (whole) {
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c) mx = fmaxf(mx, sv[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c)
+          if (kv0 + c < limit) mx = fmaxf(mx, sv[c]);
+      }
+      const float m_cand = mx == -INFINITY ? -INFINITY : mx * scale;
+      const bool need = m_cand > m + kRescaleThreshold;
+      const float alpha = need ? ex2(m - m_cand) : 1.f;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        float ov[32];
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          tmem_ld32(o_tm + c, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) ov[x] *= alpha;
+          tmem_st32(o_tm + c, ov);
+        }
+        tmem_st_wait();
+      }
+      if (need) {
+        l *= alpha;
+        m = m_cand;
+      }
+      const float mu = m == -INFINITY ? 0.f : m;
+      float rs = 0.f;
+      if (whole) {
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c) {
-          sv[c] *= scale;
-          mx = fmaxf(mx, sv[c]);
+          sv[c] = ex2(fmaf(sv[c], scale, -mu));
+          rs += sv[c];
         }
       } else {
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c) {
-          sv[c] = (kv0 + c < limit) ? sv[c] * scale : -INFINITY;
-          mx = fmaxf(mx, sv[c]);
+          sv[c] = (kv0 + c < limit) ? ex2(fmaf(sv[c], scale, -mu)) : 0.f;
+          rs += sv[c];
         }
       }
-      const float m_new = fmaxf(m, mx);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = (m == m_new) ? 1.f : ex2(m - m_use);
-      float rs = 0.f;
+      l += rs;
+      uint32_t pw[kBlockN / 2];
 #pragma unroll
-      for (int c = 0; c < kBlockN; ++c) {
-        sv[c] = ex2(sv[c] - m_use);
-        rs += sv[c];
-      }
-      l = l * alpha + rs;
-      m = m_new;
-      if (j > 0) {
-        mbar_wait(&sm.o_done, (j - 1) & 1, wc);
-        tc_fence_after();
-      }
-      // P_j (bf16, swizzled K-major rows) -> shared memory
-#pragma unroll
-      for (int ch = 0; ch < kBlockN / 8; ++ch) {
-        uint4 w;
-        w.x = pack_bf16x2(sv[ch * 8 + 0], sv[ch * 8 + 1]);
-        w.y = pack_bf16x2(sv[ch * 8 + 2], sv[ch * 8 + 3]);
-        w.z = pack_bf16x2(sv[ch * 8 + 4], sv[ch * 8 + 5]);
-        w.w = pack_bf16x2(sv[ch * 8 + 6], sv[ch * 8 + 7]);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_addr + tile_off(r, ch)), "r"(w.x),
-                     "r"(w.y), "r"(w.z), "r"(w.w)
-                     : "memory");
-      }
-      fence_proxy_async_smem();
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        float ov[32];
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          tmem_ld32(o_tmem + c, ov);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-          tmem_st32(o_tmem + c, ov);
-        }
-        tmem_st_wait();
-      }
+      for (int c = 0; c < kBlockN / 2; ++c) pw[c] = pack_bf16x2(sv[2 * c], sv[2 * c + 1]);
+      tmem_st32(s_tm, reinterpret_cast<const float*>(pw));
+      tmem_st32(s_tm + 32, reinterpret_cast<const float*>(pw + 32));
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&sm.p_full);
+      mbar_arrive(&sm.p_full[ti]);
     }
-    // ---------------------------------------------------------- epilogue
+    // ------------------------------------------------------------ epilogue
     if (n_tiles > 0) {
-      mbar_wait(&sm.o_done, (n_tiles - 1) & 1, wc);
+      mbar_wait(&sm.o_final, 0, wc);
       tc_fence_after();
     }
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const float lse2 = l > 0.f ? m + __log2f(l) : -INFINITY;
     const int tok = req.q_start + t;
     const int h = unit.kv_head * G + pr % G;
-    const int Dv = D;
     if (unit.partial >= 0) {
-      float* dst = a.dv.part_o + ((size_t)unit.partial * kBlockM + r) * Dv;
+      float* dst = a.dv.part_o + ((size_t)unit.partial * kPrefillUnitRows + ru) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         float ov[32];
         if (n_tiles > 0) {
-          tmem_ld32(o_tmem + c, ov);
+          tmem_ld32(o_tm + c, ov);
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+          for (int x = 0; x < 32; ++x) ov[x] = 0.f;
         }
         if (row_ok) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dst + c + i) =
-                make_float4(ov[i] * inv_l, ov[i + 1] * inv_l, ov[i + 2] * inv_l, ov[i + 3] * inv_l);
+          for (int x = 0; x < 32; x += 4)
+            *reinterpret_cast<float4*>(dst + c + x) =
+                make_float4(ov[x] * inv_l, ov[x + 1] * inv_l, ov[x + 2] * inv_l, ov[x + 3] * inv_l);
         }
       }
-      if (row_ok) a.dv.part_lse[(size_t)unit.partial * kBlockM + r] = lse2;
+      if (row_ok) a.dv.part_lse[(size_t)unit.partial * kPrefillUnitRows + ru] = lse2;
     } else {
-      __nv_bfloat16* dst = a.o + ((size_t)tok * a.g.num_qo_heads + h) * Dv;
+      __nv_bfloat16* dst = a.o + ((size_t)tok * a.g.num_qo_heads + h) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         float ov[32];
         if (n_tiles > 0) {
-          tmem_ld32(o_tmem + c, ov);
+          tmem_ld32(o_tm + c, ov);
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+          for (int x = 0; x < 32; ++x) ov[x] = 0.f;
         }
         if (row_ok) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
+          for (int x = 0; x < 32; x += 8) {
             uint4 w;
-            w.x = pack_bf16x2(ov[i + 0] * inv_l, ov[i + 1] * inv_l);
-            w.y = pack_bf16x2(ov[i + 2] * inv_l, ov[i + 3] * inv_l);
-            w.z = pack_bf16x2(ov[i + 4] * inv_l, ov[i + 5] * inv_l);
-            w.w = pack_bf16x2(ov[i + 6] * inv_l, ov[i + 7] * inv_l);
-            *reinterpret_cast<uint4*>(dst + c + i) = w;
+            w.x = pack_bf16x2(ov[x + 0] * inv_l, ov[x + 1] * inv_l);
+            w.y = pack_bf16x2(ov[x + 2] * inv_l, ov[x + 3] * inv_l);
+            w.z = pack_bf16x2(ov[x + 4] * inv_l, ov[x + 5] * inv_l);
+            w.w = pack_bf16x2(ov[x + 6] * inv_l, ov[x + 7] * inv_l);
+            *reinterpret_cast<uint4*>(dst + c + x) = w;
           }
         }
       }
@@ -355,23 +430,70 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor [rows][heads][D] (D contiguous), box {64, box_heads, box_rows},
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, int D, int heads, int64_t rows, int box_heads, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn || rows <= 0) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch(const Args& a, cudaStream_t stream) {
   const size_t smem = sizeof(Smem<D>) + 1024;
-  auto kern = prefill_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  kern<<<a.g.num_units, kThreads, smem, stream>>>(a);
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  prefill_kernel<D><<<a.g.num_units, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_prefill(const LaunchGeom& g, const DeviceView& dv, const int32_t* kv_indices, const void* q,
-                           const void* k, const void* v, void* o, float* lse, cudaStream_t stream) {
+                           const void* k, const void* v, int32_t num_pages, void* o, float* lse,
+                           cudaStream_t stream) {
   if (g.num_units == 0) return cudaSuccess;
-  Args a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-         static_cast<const __nv_bfloat16*>(v), kv_indices, static_cast<__nv_bfloat16*>(o), lse, g, dv};
+  Args a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.kv_indices = kv_indices;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.g = g;
+  a.dv = dv;
+  const int64_t pool_rows = (int64_t)num_pages * g.page_size;
+  a.oob_row = (int32_t)pool_rows;
+  a.q_tma = (kTileM % g.group == 0) &&
+            make_map(&a.tm_q, q, g.head_dim, g.num_qo_heads, g.total_q, g.group, kTileM / g.group);
+  a.kv_tma = g.page_size >= 8 && pool_rows < INT32_MAX &&
+             make_map(&a.tm_k, k, g.head_dim, g.num_kv_heads, pool_rows, 1, g.page_size < kBlockN ? g.page_size : kBlockN) &&
+             make_map(&a.tm_v, v, g.head_dim, g.num_kv_heads, pool_rows, 1, g.page_size < kBlockN ? g.page_size : kBlockN);
   if (g.head_dim == 128) return launch<128>(a, stream);
   if (g.head_dim == 64) return launch<64>(a, stream);
   return cudaErrorInvalidValue;
