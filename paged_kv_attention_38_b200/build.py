@@ -55,6 +55,28 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
     return obj
 
 
+def build_variant(out_lib: str, defines) -> str:
+    """Build a separate copy of the library with extra -D defines (tuning sweeps)."""
+    bdir = os.path.join(os.path.dirname(os.path.abspath(out_lib)), "_build_" + os.path.basename(out_lib))
+    os.makedirs(bdir, exist_ok=True)
+    objs = []
+    for s in SOURCES:
+        src = os.path.join(CSRC, s)
+        obj = os.path.join(bdir, s + ".o")
+        if s.endswith(".cpp"):
+            cmd = [_nvcc(), *FLAGS, "-x", "c++", "-c", src, "-o", obj]
+        else:
+            cmd = [_nvcc(), *ARCH, *FLAGS, *[f"-D{d}" for d in defines], "-c", src, "-o", obj]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"nvcc failed for {src}:\n{r.stderr}")
+        objs.append(obj)
+    r = subprocess.run([_nvcc(), *ARCH, "-shared", "-o", out_lib, *objs, "-cudart", "static"], capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(r.stderr)
+    return out_lib
+
+
 def build(verbose_ptxas: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs = [os.path.join(CSRC, s) for s in SOURCES]

@@ -54,6 +54,15 @@ constexpr int kProdWarp0 = 9;
 constexpr int kProdThreads = 96;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
+// Columns c with (c % 8) < kPolyPer8 take 2^x from the FMA-pipe polynomial,
+// the rest from MUFU ex2: the split that balances the two pipes.
+#ifndef PKV_POLY_PER8
+#define PKV_POLY_PER8 0
+#endif
+constexpr int kPolyPer8 = PKV_POLY_PER8;
+constexpr int kRegsSupport = 96;
+constexpr int kRegsSoftmax = 200;
+static_assert(128 * kRegsSupport + 256 * kRegsSoftmax <= kThreads * 168, "register split exceeds the launch budget");
 static_assert(kTileM * kTiles == kPrefillUnitRows, "unit rows");
 
 // Byte offset of 16-byte chunk `ch` of row `r` in a [128 x D] bf16 tile held as
@@ -131,7 +140,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   WaitCtx wc{&sm.abort_flag, a.dv.status};
-
+  // Registers: 384 threads x 168 at launch = 64512. The MMA/producer warpgroup
+  // (warps 8-11) drops to kRegsSupport, the two softmax warpgroups rise to
+  // kRegsSoftmax: 128 x 96 + 256 x 200 = 63488 <= 64512. Each role's code sits under its own
+  // setmaxnreg so the compiler allocates it with that budget.
+  if (warp >= kMmaWarp) {
+    setmaxnreg_dec<kRegsSupport>();
   if (warp >= kProdWarp0) {
     // ================================================================ producer
     const int pt = tid - kProdWarp0 * 32;
@@ -291,7 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       mbar_drain(&sm.o_final, 0);  // no MMA may still run when TMEM is released
     }
     __syncwarp();
+  }
   } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ================================================================ softmax
     const int ti = warp >> 2;          // query tile
     const int r = tid & (kTileM - 1);  // row in tile == TMEM lane
@@ -315,15 +331,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       tmem_ld_wait();
       const int kv0 = unit.kv_lo + j * kBlockN;
       const bool whole = kv0 + kBlockN <= limit;
-      float mx = -INFINITY;
-      if (whole) {
-#pragma unroll
-        for (int c = 0; c < kBlockN; ++c) mx = fmaxf(mx, sv[c]);
-      } else {
+      if (!whole) {
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c)
-          if (kv0 + c < limit) mx = fmaxf(mx, sv[c]);
+          if (kv0 + c >= limit) sv[c] = -INFINITY;
       }
+      // row max: four independent 3-input max chains
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < kBlockN; c += 8) {
+        mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c], sv[c + 1]);
+        mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c + 2], sv[c + 3]);
+        mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c + 4], sv[c + 5]);
+        mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c + 6], sv[c + 7]);
+      }
+      const float mx = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
       const float m_cand = mx == -INFINITY ? -INFINITY : mx * scale;
       const bool need = m_cand > m + kRescaleThreshold;
       const float alpha = need ? ex2(m - m_cand) : 1.f;
@@ -344,20 +366,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         m = m_cand;
       }
       const float mu = m == -INFINITY ? 0.f : m;
-      float rs = 0.f;
-      if (whole) {
+      // p = 2^(s * scale - m): kPolyPer8 columns in eight on the FMA pipe, the rest on MUFU.
+      // Masked columns hold -inf and give exactly 0 either way (the polynomial
+      // path is clamped, so it is zeroed explicitly).
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kBlockN; ++c) {
-          sv[c] = ex2(fmaf(sv[c], scale, -mu));
-          rs += sv[c];
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kBlockN; ++c) {
-          sv[c] = (kv0 + c < limit) ? ex2(fmaf(sv[c], scale, -mu)) : 0.f;
-          rs += sv[c];
-        }
+      for (int c = 0; c < kBlockN; ++c) {
+        const float x = fmaf(sv[c], scale, -mu);
+        float p;
+        if ((c & 7) < kPolyPer8) p = whole ? exp2_poly(x) : (sv[c] == -INFINITY ? 0.f : exp2_poly(x));
+        else p = ex2(x);
+        sv[c] = p;
+        rs4[c & 3] += p;
       }
+      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       l += rs;
       uint32_t pw[kBlockN / 2];
 #pragma unroll

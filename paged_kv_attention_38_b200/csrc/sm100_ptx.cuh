@@ -252,6 +252,39 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for use beside ex2 (the MUFU pipe is the softmax's
+// bottleneck). Round-to-nearest range reduction x = j + f, f in [-1/2, 1/2],
+// through the 1.5 * 2^23 shifter (j lands in the low mantissa bits of t), then
+// a degree-3 polynomial for 2^f and j added into the exponent field.
+// Coefficients: our own minimax fit of 2^f on [-1/2, 1/2] in relative error
+// (Lawson's iteratively reweighted least squares, then rounded to fp32);
+// max relative error 7.5e-5, far below the bf16 rounding P gets next.
+// Inputs below -126 are clamped (the result is then ~2^-126, i.e. 0 for P).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float shifter = 12582912.0f;  // 1.5 * 2^23
+  const float t = x + shifter;
+  const float j = t - shifter;
+  const float f = x - j;
+  float p = fmaf(0.0551716685f, f, 0.2426111400f);
+  p = fmaf(p, f, 0.6932609677f);
+  p = fmaf(p, f, 0.9999280572f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Raise / lower this warpgroup's per-thread register budget (all four warps of
+// the warpgroup execute it; the sum over the CTA must fit the launch budget).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
