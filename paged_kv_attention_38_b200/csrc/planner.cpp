@@ -47,6 +47,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
     *err = "page_size must be a power of two in [1, 256]"; return 2;
   }
   if (!std::isfinite(in.sm_scale)) { *err = "sm_scale is not finite"; return 1; }
+  if (!(in.sm_scale > 0.f)) { *err = "sm_scale must be positive"; return 2; }
   const int32_t group = in.num_qo_heads / in.num_kv_heads;
   if (mla) {
     if (in.num_kv_heads != 1 || in.head_dim != 512 || in.head_dim_v != 512 || in.head_dim_pe != 64) {

@@ -80,7 +80,7 @@ struct __align__(1024) Smem {
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
   uint64_t s_full[kTiles];
-  uint64_t p_full[kTiles];
+  uint64_t p_half[kTiles][2];  // P_i columns [0,64) / [64,128) written
   uint64_t o_final;
   int32_t rowsrc[kBlockN];  // cp.async gather: pool row of each tile row, -1 = zero fill
   uint32_t tmem_base;
@@ -125,7 +125,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     }
     for (int i = 0; i < kTiles; ++i) {
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i], kTileM);
+      mbar_init(&sm.p_half[i][0], kTileM);
+      mbar_init(&sm.p_half[i][1], kTileM);
     }
     mbar_init(&sm.o_final, 1);
     sm.abort_flag = 0;
@@ -266,10 +267,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                     idesc_s, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int i, int j) {
+      // O_i += P_i V_j for kv columns [32h, 32h + 64) of this tile: K-steps 4h..4h+3.
+      auto issue_pv_half = [&](int i, int j, int h) {
         const uint32_t v_addr = smem_u32(sm.kv[(2 * j + 1) & (kSlots - 1)]);
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk)
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
           umma_bf16_ts(tmem + 256 + i * 128, tmem + i * kBlockN + kk * 8,
                        sdesc_sw128(v_addr + kk * 16 * 128, kBlockN * 128, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
       };
@@ -283,17 +285,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       umma_commit(&sm.empty[0]);
       for (int j = 0; j < n_tiles; ++j) {
         const bool more = j + 1 < n_tiles;
-        mbar_wait(&sm.p_full[0], j & 1, wc);
+        mbar_wait(&sm.p_half[0][0], j & 1, wc);
         wait_item(2 * j + 1);
-        issue_pv(0, j);
+        issue_pv_half(0, j, 0);
+        mbar_wait(&sm.p_half[0][1], j & 1, wc);
+        tc_fence_after();
+        issue_pv_half(0, j, 1);
         if (more) {
           wait_item(2 * j + 2);
           issue_s(0, j + 1);
           umma_commit(&sm.s_full[0]);
         }
-        mbar_wait(&sm.p_full[1], j & 1, wc);
+        mbar_wait(&sm.p_half[1][0], j & 1, wc);
         tc_fence_after();
-        issue_pv(1, j);
+        issue_pv_half(1, j, 0);
+        mbar_wait(&sm.p_half[1][1], j & 1, wc);
+        tc_fence_after();
+        issue_pv_half(1, j, 1);
         umma_commit(&sm.empty[(2 * j + 1) & (kSlots - 1)]);
         if (more) {
           issue_s(1, j + 1);
@@ -366,29 +374,44 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         m = m_cand;
       }
       const float mu = m == -INFINITY ? 0.f : m;
-      // p = 2^(s * scale - m): kPolyPer8 columns in eight on the FMA pipe, the rest on MUFU.
-      // Masked columns hold -inf and give exactly 0 either way (the polynomial
-      // path is clamped, so it is zeroed explicitly).
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      // p = 2^(s * scale - m) (masked columns hold -inf and give 0), packed to
+      // bf16 and stored over S in 32-column chunks; each half of P is published
+      // as soon as it is in TMEM so the P.V MMAs can start on it.
+      const float2 scale2 = make_float2(scale, scale);
+      const float2 nmu2 = make_float2(-mu, -mu);
+      float2 rs2a = make_float2(0.f, 0.f), rs2b = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < kBlockN; ++c) {
-        const float x = fmaf(sv[c], scale, -mu);
-        float p;
-        if ((c & 7) < kPolyPer8) p = whole ? exp2_poly(x) : (sv[c] == -INFINITY ? 0.f : exp2_poly(x));
-        else p = ex2(x);
-        sv[c] = p;
-        rs4[c & 3] += p;
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c0 = h * 64 + cc * 32;
+          uint32_t pw[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float2 x = ffma2(make_float2(sv[c0 + 2 * e], sv[c0 + 2 * e + 1]), scale2, nmu2);
+            float2 pp;
+            if (kPolyPer8 > 0 && ((2 * e) & 7) < kPolyPer8) {
+              pp.x = exp2_poly(x.x);
+              pp.y = exp2_poly(x.y);
+              if (!whole) {
+                if (sv[c0 + 2 * e] == -INFINITY) pp.x = 0.f;
+                if (sv[c0 + 2 * e + 1] == -INFINITY) pp.y = 0.f;
+              }
+            } else {
+              pp.x = ex2(x.x);
+              pp.y = ex2(x.y);
+            }
+            if (e & 1) rs2b = fadd2(rs2b, pp);
+            else rs2a = fadd2(rs2a, pp);
+            pw[e] = pack_bf16x2(pp.x, pp.y);
+          }
+          tmem_st16(s_tm + h * 32 + cc * 16, pw);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sm.p_half[ti][h]);
       }
-      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-      l += rs;
-      uint32_t pw[kBlockN / 2];
-#pragma unroll
-      for (int c = 0; c < kBlockN / 2; ++c) pw[c] = pack_bf16x2(sv[2 * c], sv[2 * c + 1]);
-      tmem_st32(s_tm, reinterpret_cast<const float*>(pw));
-      tmem_st32(s_tm + 32, reinterpret_cast<const float*>(pw + 32));
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&sm.p_full[ti]);
+      l += (rs2a.x + rs2a.y) + (rs2b.x + rs2b.y);
     }
     // ------------------------------------------------------------ epilogue
     if (n_tiles > 0) {

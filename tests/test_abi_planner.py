@@ -166,6 +166,7 @@ def test_longest_units_first():
     (lambda a: a.__setitem__("d", 96), pkv.PKV_EUNSUPPORTED),          # unsupported head_dim
     (lambda a: a.__setitem__("hk", 3), pkv.PKV_EINVAL),                # hq % hk != 0
     (lambda a: a.__setitem__("scale", float("nan")), pkv.PKV_EINVAL),  # sm_scale not finite
+    (lambda a: a.__setitem__("scale", 0.0), pkv.PKV_EUNSUPPORTED),     # sm_scale must be positive
 ])
 def test_error_codes(mutate, status):
     a = dict(qo=np.array([0, 5, 9], np.int32), kv=np.array([0, 1, 2], np.int32),
