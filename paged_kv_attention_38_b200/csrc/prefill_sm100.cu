@@ -257,23 +257,31 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         fence_proxy_async_smem();  // cp.async rows were written through the generic proxy
         tc_fence_after();
       };
+      // Descriptors are built once; a K-step only moves the start address,
+      // which is the low 14-bit field (addr >> 4), so it is added in place.
+      uint64_t dq[kTiles], dk[kSlots], dv[kSlots];
+#pragma unroll
+      for (int i = 0; i < kTiles; ++i) dq[i] = sdesc_sw128(smem_u32(sm.q[i]), 16, 1024);
+#pragma unroll
+      for (int sl = 0; sl < kSlots; ++sl) {
+        dk[sl] = sdesc_sw128(smem_u32(sm.kv[sl]), 16, 1024);
+        dv[sl] = sdesc_sw128(smem_u32(sm.kv[sl]), kBlockN * 128, 1024);
+      }
       auto issue_s = [&](int i, int j) {
-        const uint32_t k_addr = smem_u32(sm.kv[(2 * j) & (kSlots - 1)]);
-        const uint32_t q_addr = smem_u32(sm.q[i]);
+        const uint64_t bq = dq[i], bk = dk[(2 * j) & (kSlots - 1)];
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTileM * 128) + (kk & 3) * 32;
-          umma_bf16(tmem + i * kBlockN, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
-                    idesc_s, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
+          umma_bf16(tmem + i * kBlockN, bq + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
         }
       };
-      // O_i += P_i V_j for kv columns [32h, 32h + 64) of this tile: K-steps 4h..4h+3.
+      // O_i += P_i V_j for kv columns [64h, 64h + 64) of this tile: K-steps 4h..4h+3.
       auto issue_pv_half = [&](int i, int j, int h) {
-        const uint32_t v_addr = smem_u32(sm.kv[(2 * j + 1) & (kSlots - 1)]);
+        const uint64_t bv = dv[(2 * j + 1) & (kSlots - 1)];
 #pragma unroll
         for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
-          umma_bf16_ts(tmem + 256 + i * 128, tmem + i * kBlockN + kk * 8,
-                       sdesc_sw128(v_addr + kk * 16 * 128, kBlockN * 128, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + 256 + i * 128, tmem + i * kBlockN + kk * 8, bv + ((kk * 16 * 128) >> 4), idesc_o,
+                       (j > 0 || kk > 0) ? 1u : 0u);
       };
       mbar_wait(&sm.q_full, 0, wc);
       fence_proxy_async_smem();
@@ -334,8 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       mbar_wait(&sm.s_full[ti], j & 1, wc);
       tc_fence_after();
       float sv[kBlockN];
-#pragma unroll
-      for (int c = 0; c < kBlockN; c += 32) tmem_ld32(s_tm + c, sv + c);
+      tmem_ld64(s_tm, sv);
+      tmem_ld64(s_tm + 64, sv + 64);
       tmem_ld_wait();
       const int kv0 = unit.kv_lo + j * kBlockN;
       const bool whole = kv0 + kBlockN <= limit;
@@ -382,31 +390,27 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       float2 rs2a = make_float2(0.f, 0.f), rs2b = make_float2(0.f, 0.f);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
+        uint32_t pw[32];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c0 = h * 64 + cc * 32;
-          uint32_t pw[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float2 x = ffma2(make_float2(sv[c0 + 2 * e], sv[c0 + 2 * e + 1]), scale2, nmu2);
-            float2 pp;
-            if (kPolyPer8 > 0 && ((2 * e) & 7) < kPolyPer8) {
-              pp.x = exp2_poly(x.x);
-              pp.y = exp2_poly(x.y);
-              if (!whole) {
-                if (sv[c0 + 2 * e] == -INFINITY) pp.x = 0.f;
-                if (sv[c0 + 2 * e + 1] == -INFINITY) pp.y = 0.f;
-              }
-            } else {
-              pp.x = ex2(x.x);
-              pp.y = ex2(x.y);
+        for (int e = 0; e < 32; ++e) {
+          const int c = h * 64 + 2 * e;
+          const float2 x = ffma2(make_float2(sv[c], sv[c + 1]), scale2, nmu2);
+          float2 pp;
+          if (kPolyPer8 > 0 && ((2 * e) & 7) < kPolyPer8) {
+            pp = exp2_poly2(x);
+            if (!whole) {
+              if (sv[c] == -INFINITY) pp.x = 0.f;
+              if (sv[c + 1] == -INFINITY) pp.y = 0.f;
             }
-            if (e & 1) rs2b = fadd2(rs2b, pp);
-            else rs2a = fadd2(rs2a, pp);
-            pw[e] = pack_bf16x2(pp.x, pp.y);
+          } else {
+            pp.x = ex2(x.x);
+            pp.y = ex2(x.y);
           }
-          tmem_st16(s_tm + h * 32 + cc * 16, pw);
+          if (e & 1) rs2b = fadd2(rs2b, pp);
+          else rs2a = fadd2(rs2a, pp);
+          pw[e] = pack_bf16x2(pp.x, pp.y);
         }
+        tmem_st32(s_tm + h * 32, reinterpret_cast<const float*>(pw));
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sm.p_half[ti][h]);
