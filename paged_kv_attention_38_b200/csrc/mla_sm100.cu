@@ -1,13 +1,358 @@
-// Absorbed-MLA paged prefill (placeholder until the tcgen05 kernel lands).
+// Absorbed-MLA paged prefill on sm_100a tensor cores.
+//
+// What it computes (FlashInfer 0.2 release, "Fused MLA decode kernel" and its
+// matrix-absorption trick; definition mla_paged_prefill_causal_h16_ckv512_kpe64_ps1
+// in flashinfer-trace discussion #15): all H query heads share one latent KV
+// row per token, the compressed ckv (512) and the rope key kpe (64). With the
+// projections absorbed into the query and output,
+//   s_j = sm_scale * (q_nope . ckv_j + q_pe . kpe_j),   o = sum_j softmax(s)_j ckv_j,
+// i.e. attention with a 576-wide key [ckv | kpe] and a 512-wide value ckv.
+// Output O (bf16, 512 per head) and the base-2 LSE per (token, head).
+//
+// Shape choices for B200. A 128-row tile's 128 x 512 fp32 output alone would
+// fill all 512 TMEM columns, and a 128 x 576 bf16 query tile (144 KB) leaves no
+// room in shared memory for a double-buffered key tile. So a CTA takes 64
+// packed (token, head) rows and 64-key tiles, and runs M = 64 MMAs:
+//   TMEM  O rows x latent[0,256)   lanes 16q + [0,16)  (q = sub-partition), cols [0,256)
+//         O rows x latent[256,512) lanes 16q + [16,32),                     cols [0,256)
+//         S (double buffer)        lanes 16q + [0,16),                      cols [256,320), [320,384)
+//   (a 64-row accumulator uses half of each 32-lane sub-partition; the two
+//   latent halves of O sit in the two halves, so a warp rescales both with one
+//   32x32b load/store over columns [0,256) without touching S.)
+//   SMEM  Q 64 x 576 (72 KB), a 2-stage ring of 64 x 576 latent rows (K and V
+//   at once: V is the ckv part of the same rows), P 64 x 64 (8 KB).
+// Both MMAs read their operands from shared memory. Warps: 0-3 softmax and
+// epilogue (lanes 0-15 own S rows and the low O half, lanes 16-31 the high O
+// half of the same rows), 4 TMEM allocator + MMA issuer, 5-8 cp.async gather
+// of Q and of the latent rows through the page table.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "pkv_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace pkv {
 
-cudaError_t launch_mla(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
-                       const void*, const void*, void*, float*, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int kRows = kMlaUnitRows;  // 64
+constexpr int kN = 64;               // keys per tile
+constexpr int kDc = 512;
+constexpr int kDr = 64;
+constexpr int kDqk = kDc + kDr;      // 576
+constexpr int kBlocks = kDqk / 64;   // 9 column blocks of 64 (128-byte rows)
+constexpr int kBlockBytes = kRows * 128;  // one [64 rows x 64] bf16 block: 8 KB
+constexpr int kThreads = 288;
+constexpr int kMmaWarp = 4;
+constexpr int kProdWarp0 = 5;
+constexpr int kProdThreads = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSCol = 256;
+constexpr float kRescaleThreshold = 8.0f;
+static_assert(kN == kRows, "one block shape for Q, latent rows and P");
+
+// Byte offset of 16-byte chunk `ch` (0..71 across the 576-wide row) of row `r`
+// in a [64 x 576] tile held as 9 column blocks of [64 rows x 128 B], 128-byte swizzle.
+__device__ __forceinline__ uint32_t blk_off(int r, int ch) {
+  return (uint32_t)((ch >> 3) * kBlockBytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+}
+
+struct __align__(1024) Smem {
+  __nv_bfloat16 q[kBlocks * kRows * 64];
+  __nv_bfloat16 kv[2][kBlocks * kN * 64];
+  __nv_bfloat16 p[kRows * kN];
+  uint64_t q_full;
+  uint64_t kv_full[2];
+  uint64_t kv_empty[2];
+  uint64_t s_full[2];
+  uint64_t s_free[2];
+  uint64_t p_full;
+  uint64_t o_done;
+  uint64_t o_final;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct Args {
+  const __nv_bfloat16* q_nope;
+  const __nv_bfloat16* q_pe;
+  const __nv_bfloat16* ckv;
+  const __nv_bfloat16* kpe;
+  const int32_t* kv_indices;
+  __nv_bfloat16* o;
+  float* lse;
+  LaunchGeom g;
+  DeviceView dv;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant__ Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const WorkUnit unit = a.dv.units[blockIdx.x];
+  const ReqInfo req = a.dv.reqs[unit.req];
+  const int H = a.g.num_qo_heads;
+  const int n_tiles = (unit.kv_hi - unit.kv_lo + kN - 1) / kN;
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, kProdThreads);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.kv_full[s], kProdThreads);
+      mbar_init(&sm.kv_empty[s], 1);
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.s_free[s], 128);
+    }
+    mbar_init(&sm.p_full, 128);
+    mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.o_final, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  WaitCtx wc{&sm.abort_flag, a.dv.status};
+
+  if (warp >= kProdWarp0) {
+    // ================================================================ producer
+    const int pt = tid - kProdWarp0 * 32;
+    constexpr int kChunks = kDqk / 8;  // 72 16-byte chunks per 576-wide row
+    const int P = a.g.page_size, shift = a.g.page_shift;
+    if (n_tiles > 0) {
+      for (int c = pt; c < kRows * kChunks; c += kProdThreads) {
+        const int r = c / kChunks, ch = c % kChunks;
+        const bool ok = r < unit.rows;
+        const __nv_bfloat16* src = a.q_nope;
+        if (ok) {
+          const int pr = unit.row0 + r;
+          const size_t row = (size_t)(req.q_start + pr / H) * H + pr % H;
+          src = ch < kDc / 8 ? a.q_nope + row * kDc + ch * 8 : a.q_pe + row * kDr + (ch - kDc / 8) * 8;
+        }
+        cp_async_16(smem_u32(sm.q) + blk_off(r, ch), src, ok ? 16u : 0u);
+      }
+      cp_async_arrive_noinc(&sm.q_full);
+    }
+    for (int j = 0; j < n_tiles; ++j) {
+      const int st = j & 1;
+      if (j >= 2) mbar_wait(&sm.kv_empty[st], ((j >> 1) - 1) & 1, wc);
+      const uint32_t dst = smem_u32(sm.kv[st]);
+      for (int c = pt; c < kN * kChunks; c += kProdThreads) {
+        const int r = c / kChunks, ch = c % kChunks;
+        const int pos = unit.kv_lo + j * kN + r;
+        const bool ok = pos < unit.kv_hi;
+        const __nv_bfloat16* src = a.ckv;
+        if (ok) {
+          const size_t slot = (size_t)__ldg(a.kv_indices + req.page0 + (pos >> shift)) * P + (pos & (P - 1));
+          src = ch < kDc / 8 ? a.ckv + slot * kDc + ch * 8 : a.kpe + slot * kDr + (ch - kDc / 8) * 8;
+        }
+        cp_async_16(dst + blk_off(r, ch), src, ok ? 16u : 0u);
+      }
+      cp_async_arrive_noinc(&sm.kv_full[st]);
+    }
+    cp_async_wait<0>();
+  } else if (warp == kMmaWarp) {
+    // ================================================================ MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kRows, kN, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kRows, 256, true);
+      const uint64_t dq = sdesc_sw128(smem_u32(sm.q), 16, 1024);
+      const uint64_t dp = sdesc_sw128(smem_u32(sm.p), 16, 1024);
+      uint64_t dk[2], dvv[2];
+      for (int s = 0; s < 2; ++s) {
+        dk[s] = sdesc_sw128(smem_u32(sm.kv[s]), 16, 1024);
+        dvv[s] = sdesc_sw128(smem_u32(sm.kv[s]), kBlockBytes, 1024);
+      }
+      auto issue_pv = [&](int jj) {
+        const int st = jj & 1;
+        mbar_wait(&sm.p_full, jj & 1, wc);
+        fence_proxy_async_smem();
+        tc_fence_after();
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+          const uint32_t d = tmem + (nh ? (16u << 16) : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kN / 16; ++kk)
+            umma_bf16(d, dp + ((kk * 32) >> 4), dvv[st] + ((4 * nh * kBlockBytes + kk * 16 * 128) >> 4), idesc_o,
+                      (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&sm.o_done);
+        umma_commit(&sm.kv_empty[st]);
+      };
+      mbar_wait(&sm.q_full, 0, wc);
+      for (int j = 0; j < n_tiles; ++j) {
+        const int st = j & 1;
+        mbar_wait(&sm.kv_full[st], (j >> 1) & 1, wc);
+        if (j >= 2) mbar_wait(&sm.s_free[st], ((j >> 1) - 1) & 1, wc);
+        fence_proxy_async_smem();  // cp.async rows were written through the generic proxy
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kDqk / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4;
+          umma_bf16(tmem + kSCol + st * kN, dq + off, dk[st] + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&sm.s_full[st]);
+        if (j >= 1) issue_pv(j - 1);
+      }
+      issue_pv(n_tiles - 1);
+      umma_commit(&sm.o_final);
+      mbar_drain(&sm.o_final, 0);
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ softmax
+    const bool s_owner = lane < 16;
+    const int row = warp * 16 + (lane & 15);  // row of the unit this thread's S / O half belongs to
+    const bool row_ok = row < unit.rows;
+    const int pr = unit.row0 + (row_ok ? row : 0);
+    const int t = pr / H;
+    int limit = unit.kv_hi;
+    if (a.g.causal) limit = min(limit, t + req.kv_len - req.qo_len + 1);
+    const float scale = a.g.sm_scale_log2;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float m = -INFINITY, l = 0.f;
+    const uint32_t p_addr = smem_u32(sm.p);
+    for (int j = 0; j < n_tiles; ++j) {
+      const int st = j & 1;
+      mbar_wait(&sm.s_full[st], (j >> 1) & 1, wc);
+      tc_fence_after();
+      float sv[kN];
+      tmem_ld32(lane_base + kSCol + st * kN, sv);
+      tmem_ld32(lane_base + kSCol + st * kN + 32, sv + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&sm.s_free[st]);
+      const int kv0 = unit.kv_lo + j * kN;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kN; ++c) {
+        if (kv0 + c >= limit) sv[c] = -INFINITY;
+        mx = fmaxf(mx, sv[c]);
+      }
+      const float m_cand = mx == -INFINITY ? -INFINITY : mx * scale;
+      bool need = s_owner && m_cand > m + kRescaleThreshold;
+      float alpha = need ? ex2(m - m_cand) : 1.f;
+      // the high-half O row of lane 16 + i belongs to the S row of lane i
+      const float alpha_o = __shfl_sync(0xffffffffu, alpha, lane & 15);
+      const bool any = __any_sync(0xffffffffu, need);
+      if (j > 0) {
+        mbar_wait(&sm.o_done, (j - 1) & 1, wc);  // P buffer free, O stable
+        tc_fence_after();
+        if (any) {
+          float ov[32];
+#pragma unroll 1
+          for (int c = 0; c < 256; c += 32) {
+            tmem_ld32(lane_base + c, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) ov[x] *= alpha_o;
+            tmem_st32(lane_base + c, ov);
+          }
+          tmem_st_wait();
+        }
+      }
+      if (need) {
+        l *= alpha;
+        m = m_cand;
+      }
+      if (s_owner) {
+        const float mu = m == -INFINITY ? 0.f : m;
+        float rs = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < kN / 8; ++ch) {
+          float pv[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            pv[x] = ex2(fmaf(sv[ch * 8 + x], scale, -mu));
+            rs += pv[x];
+          }
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_addr + row * 128 + ((ch ^ (row & 7)) << 4)),
+                       "r"(pack_bf16x2(pv[0], pv[1])), "r"(pack_bf16x2(pv[2], pv[3])),
+                       "r"(pack_bf16x2(pv[4], pv[5])), "r"(pack_bf16x2(pv[6], pv[7]))
+                       : "memory");
+        }
+        l += rs;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (n_tiles > 0) {
+      mbar_wait(&sm.o_final, 0, wc);
+      tc_fence_after();
+    }
+    const float l_row = __shfl_sync(0xffffffffu, l, lane & 15);
+    const float m_row = __shfl_sync(0xffffffffu, m, lane & 15);
+    const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+    const float lse2 = l_row > 0.f ? m_row + __log2f(l_row) : -INFINITY;
+    const int half = s_owner ? 0 : 1;
+    const size_t orow = (size_t)(req.q_start + t) * H + pr % H;
+    for (int c = 0; c < 256; c += 32) {
+      float ov[32];
+      if (n_tiles > 0) {
+        tmem_ld32(lane_base + c, ov);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int x = 0; x < 32; ++x) ov[x] = 0.f;
+      }
+      if (!row_ok) continue;
+      const int d0 = half * 256 + c;
+      if (unit.partial >= 0) {
+        float* dst = a.dv.part_o + ((size_t)unit.partial * kRows + row) * kDc + d0;
+#pragma unroll
+        for (int x = 0; x < 32; x += 4)
+          *reinterpret_cast<float4*>(dst + x) =
+              make_float4(ov[x] * inv_l, ov[x + 1] * inv_l, ov[x + 2] * inv_l, ov[x + 3] * inv_l);
+      } else {
+        __nv_bfloat16* dst = a.o + orow * kDc + d0;
+#pragma unroll
+        for (int x = 0; x < 32; x += 8) {
+          uint4 w;
+          w.x = pack_bf16x2(ov[x + 0] * inv_l, ov[x + 1] * inv_l);
+          w.y = pack_bf16x2(ov[x + 2] * inv_l, ov[x + 3] * inv_l);
+          w.z = pack_bf16x2(ov[x + 4] * inv_l, ov[x + 5] * inv_l);
+          w.w = pack_bf16x2(ov[x + 6] * inv_l, ov[x + 7] * inv_l);
+          *reinterpret_cast<uint4*>(dst + x) = w;
+        }
+      }
+    }
+    if (row_ok && s_owner) {
+      if (unit.partial >= 0) a.dv.part_lse[(size_t)unit.partial * kRows + row] = lse2;
+      else if (a.lse) a.lse[orow] = lse2;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+cudaError_t launch_mla(const LaunchGeom& g, const DeviceView& dv, const int32_t* kv_indices, const void* q_nope,
+                       const void* q_pe, const void* ckv, const void* kpe, void* o, float* lse,
+                       cudaStream_t stream) {
+  if (g.num_units == 0) return cudaSuccess;
+  Args a{static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_pe),
+         static_cast<const __nv_bfloat16*>(ckv), static_cast<const __nv_bfloat16*>(kpe), kv_indices,
+         static_cast<__nv_bfloat16*>(o), lse, g, dv};
+  const size_t smem = sizeof(Smem) + 1024;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  mla_kernel<<<g.num_units, kThreads, smem, stream>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace pkv

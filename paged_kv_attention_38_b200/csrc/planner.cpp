@@ -93,7 +93,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   // tile; prefill units hold two 128-row tensor-core tiles that share K/V; MLA
   // packs tokens x heads the same way with one latent "kv head".
   const int32_t rows_per_tile = s.kind == kKindDecode ? kDecodeRows
-                                : s.kind == kKindMla  ? kBlockM
+                                : s.kind == kKindMla  ? kMlaUnitRows
                                                       : kPrefillUnitRows;
 
   // ---- tiles
@@ -117,7 +117,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   }
 
   // ---- split-KV chunk
-  const int32_t align = s.kind == kKindDecode ? kDecodeTileN : kBlockN;
+  const int32_t align = s.kind == kKindDecode ? kDecodeTileN : s.kind == kKindMla ? 64 : kBlockN;
   int64_t chunk = 0;  // 0 = no split
   if (!in.disable_split_kv) {
     if (in.kv_chunk > 0) {

@@ -236,3 +236,63 @@ def test_merge_state_kernels():
     ob16, l16 = pkv.merge_states(parts.cuda(), lses.cuda())
     o_ref, l_ref = oracle.merge_states(list(parts.numpy()), list(lses.numpy()))
     assert_parity(ob16, l16, o_ref, l_ref, what="merge_states")
+
+
+# --------------------------------------------------------------------------- MLA
+
+def gpu_run_mla(p: W.PagedProblem, **plan_kw):
+    d = to_dev(p)
+    pl = pkv.plan_mla(p.qo_indptr, p.kv_indptr, d["kv_indices"], p.kv_last_page_len, p.num_qo_heads, 512, 64,
+                      p.page_size, p.causal, p.sm_scale, **plan_kw)
+    o, lse = pkv.run_mla(pl, d["q_nope"], d["q_pe"], d["ckv_cache"], d["kpe_cache"])
+    torch.cuda.synchronize()
+    assert pkv.device_status(pl) == 0
+    return o, lse, pl
+
+
+def oracle_mla(p: W.PagedProblem):
+    return oracle.mla_paged_attention(p.q_nope, p.q_pe, p.ckv_cache, p.kpe_cache, p.qo_indptr, p.kv_indptr,
+                                      p.kv_indices, p.kv_last_page_len, p.page_size, p.causal, p.sm_scale)
+
+
+MLA_SWEEP = [
+    # qo_lens, kv_lens, heads, page, causal
+    ([7, 33], [7, 33], 16, 1, True),
+    ([64, 130, 1], [64, 130, 1], 16, 1, True),
+    ([40, 9], [100, 9], 16, 16, True),      # chunked prefill: qo < kv
+    ([5, 3], [3, 0], 8, 1, True),           # qo > kv (rows with no key) and an empty request
+    ([17, 80], [200, 80], 4, 4, False),
+]
+
+
+@pytest.mark.parametrize("case", MLA_SWEEP, ids=lambda c: f"q{sum(c[0])}_h{c[2]}_p{c[3]}_c{int(c[4])}")
+def test_mla_sweep(case):
+    qo, kv, h, ps, causal = case
+    p = W.make_mla_problem("mla", qo, kv, num_heads=h, page_size=ps, causal=causal,
+                           seed=zlib.crc32(str(case).encode()) % 10000)
+    o, lse, pl = gpu_run_mla(p)
+    assert pl.kind == pkv.KIND_MLA
+    assert_parity(o, lse, *oracle_mla(p), what=f"mla {case}")
+
+
+def test_mla_split_kv():
+    p = W.make_mla_problem("mla_split", [30, 200], [700, 200], num_heads=16, page_size=1, causal=True, seed=12)
+    o, lse, pl = gpu_run_mla(p, kv_chunk=128)
+    assert pl.num_merges > 0
+    assert_parity(o, lse, *oracle_mla(p), what="mla split")
+
+
+@pytest.mark.slow
+def test_mla_full_size_sampled():
+    """h16/ckv512/kpe64/ps1, batch 4, lengths U[256, 2048]: sampled rows of every request."""
+    p = W.mla_prefill()
+    o, lse, _ = gpu_run_mla(p)
+    rng = np.random.default_rng(2)
+    for b in range(p.batch):
+        L = int(p.qo_lens[b])
+        pos = sorted({0, 1, 63, 64, L - 1, *rng.integers(0, L, 3).tolist()})
+        o_r, l_r = oracle.mla_paged_attention_rows(p.q_nope, p.q_pe, p.ckv_cache, p.kpe_cache, p.qo_indptr,
+                                                   p.kv_indptr, p.kv_indices, p.kv_last_page_len, 1, True,
+                                                   p.sm_scale, b, pos)
+        rows = [int(p.qo_indptr[b]) + x for x in pos]
+        assert_parity(o[rows], lse[rows], o_r, l_r, what=f"mla req {b}")
