@@ -148,6 +148,32 @@ PKV_API pkv_status pkv_merge_state(const float* o_a, const float* lse_a, const f
 PKV_API pkv_status pkv_merge_states(const float* o_parts, const float* lse_parts, int32_t num, int32_t rows,
                             int32_t dim, void* o_out, float* lse_out, void* stream);
 
+/* Paged decode (one query token per request) for callers that cannot allocate
+ * device memory: code under an allocator that forbids new device allocations
+ * (a fixed pool, an embedded host that only registers buffers at start-up) or
+ * a serving thread that must not enter the allocator. It needs no plan and no
+ * workspace: the page table is read on the device, nothing is uploaded, and
+ * split-KV partial states live in one fixed 16 MiB device array inside the
+ * library (allocated when the library is loaded, held by every GPU that loads
+ * it until exit). The pages this library follows have no counterpart of this
+ * call; it computes the same result as pkv_run on a decode plan.
+ *   q [batch, num_qo_heads, head_dim], k_cache / v_cache as for pkv_run,
+ *   kv_indptr [batch+1], kv_indices, kv_last_page_len [batch]: all DEVICE int32.
+ *   max_kv_len: an upper bound on the requests' kv_len, used to size the split
+ *   (a larger kv_len is still computed exactly, only more slowly).
+ *   o [batch, num_qo_heads, head_dim] bf16, lse [batch, num_qo_heads] fp32 (or NULL).
+ * Supports num_qo_heads / num_kv_heads <= 16, head_dim 64 or 128.
+ * Returns PKV_ENOSPACE, without launching anything, when the split would need
+ * more than the 16 MiB of scratch. The first call on each device looks up the
+ * scratch address (cudaGetSymbolAddress) and should come before any stream
+ * capture. All calls share the scratch: calls whose kernels overlap on the GPU
+ * (other streams, unordered threads) race on it and must be serialised. */
+PKV_API pkv_status pkv_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* kv_indptr, const int32_t* kv_indices,
+                                      const int32_t* kv_last_page_len, int32_t batch, int32_t num_qo_heads,
+                                      int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
+                                      int32_t max_kv_len, float sm_scale, void* o, float* lse, void* stream);
+
 /* Read the device status word of the plan's workspace (synchronises `stream`).
  * PKV_OK if no kernel reported an error; PKV_EDEVICE otherwise (and the code is
  * stored in *code if code != NULL). */

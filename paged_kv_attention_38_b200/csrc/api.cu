@@ -112,6 +112,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 }  // namespace
 
+namespace pkv {
+// Lets other translation units of the library report through pkv_last_error().
+void set_last_error(const std::string& msg) { g_err = msg; }
+}  // namespace pkv
+
 extern "C" {
 
 pkv_status pkv_plan_create(const int32_t* qo_indptr, const int32_t* kv_indptr, const int32_t* kv_indices,
