@@ -7,7 +7,7 @@
 #include <new>
 #include <string>
 
-#include "../../include/pkv.h"
+#include "pkv.h"
 #include "pkv_internal.h"
 #include "planner.h"
 

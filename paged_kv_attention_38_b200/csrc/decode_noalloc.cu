@@ -34,7 +34,7 @@
 #include <atomic>
 #include <string>
 
-#include "../../include/pkv.h"
+#include "pkv.h"
 #include "pkv_internal.h"
 #include "sm100_ptx.cuh"
 

@@ -69,6 +69,7 @@ struct __align__(1024) Smem {
   uint64_t p_full;
   uint64_t o_done;
   uint64_t o_final;
+  int32_t rowsrc[2][kN];  // pool slot of each latent row of the tile in each stage, -1 = zero fill
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -139,20 +140,36 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
       }
       cp_async_arrive_noinc(&sm.q_full);
     }
+    // Latent tiles: the page lookups of a tile are done once (one row per
+    // thread) into shared memory; then each thread copies a fixed 16-byte
+    // column of every other row: ckv columns 0..63 (two rows per pass), kpe
+    // columns 64..71 (sixteen rows per pass).
     for (int j = 0; j < n_tiles; ++j) {
       const int st = j & 1;
       if (j >= 2) mbar_wait(&sm.kv_empty[st], ((j >> 1) - 1) & 1, wc);
+      if (pt < kN) {
+        const int pos = unit.kv_lo + j * kN + pt;
+        sm.rowsrc[st][pt] = pos < unit.kv_hi ? __ldg(a.kv_indices + req.page0 + (pos >> shift)) * P + (pos & (P - 1)) : -1;
+      }
+      named_bar_sync(1, kProdThreads);
       const uint32_t dst = smem_u32(sm.kv[st]);
-      for (int c = pt; c < kN * kChunks; c += kProdThreads) {
-        const int r = c / kChunks, ch = c % kChunks;
-        const int pos = unit.kv_lo + j * kN + r;
-        const bool ok = pos < unit.kv_hi;
-        const __nv_bfloat16* src = a.ckv;
-        if (ok) {
-          const size_t slot = (size_t)__ldg(a.kv_indices + req.page0 + (pos >> shift)) * P + (pos & (P - 1));
-          src = ch < kDc / 8 ? a.ckv + slot * kDc + ch * 8 : a.kpe + slot * kDr + (ch - kDc / 8) * 8;
+      {
+        const int ch = pt & 63;
+        const uint32_t col = (uint32_t)((ch >> 3) * kBlockBytes + ((ch & 7) << 4));
+        for (int r = pt >> 6; r < kN; r += 2) {
+          const int src = sm.rowsrc[st][r];
+          const __nv_bfloat16* g = src >= 0 ? a.ckv + (size_t)src * kDc + ch * 8 : a.ckv;
+          cp_async_16(dst + r * 128 + (col ^ ((r & 7) << 4)), g, src >= 0 ? 16u : 0u);
         }
-        cp_async_16(dst + blk_off(r, ch), src, ok ? 16u : 0u);
+      }
+      {
+        const int ch = pt & 7;
+        const uint32_t col = (uint32_t)(8 * kBlockBytes + (ch << 4));
+        for (int r = pt >> 3; r < kN; r += 16) {
+          const int src = sm.rowsrc[st][r];
+          const __nv_bfloat16* g = src >= 0 ? a.kpe + (size_t)src * kDr + ch * 8 : a.kpe;
+          cp_async_16(dst + r * 128 + (col ^ ((r & 7) << 4)), g, src >= 0 ? 16u : 0u);
+        }
       }
       cp_async_arrive_noinc(&sm.kv_full[st]);
     }

@@ -104,7 +104,10 @@ struct Args {
   int32_t oob_row;    // a pool row index past the end: TMA zero-fills it
 };
 
-template <int D>
+// kRows: K/V arrive as single rows by cp.async (page_size < 8) instead of whole
+// pages by TMA. A template parameter, so each instance holds only its own
+// producer code (the instances' register allocation is then independent).
+template <int D, bool kRows>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Args a) {
   extern __shared__ uint8_t smem_raw[];
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -120,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   if (tid == 0) {
     mbar_init(&sm.q_full, a.q_tma ? 1 : kProdThreads);
     for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&sm.full[s], a.kv_tma ? 1 : kProdThreads);
+      mbar_init(&sm.full[s], (!kRows && a.kv_tma) ? 1 : kProdThreads);
       mbar_init(&sm.empty[s], 1);
     }
     for (int i = 0; i < kTiles; ++i) {
@@ -154,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const int P = a.g.page_size, shift = a.g.page_shift, Hk = a.g.num_kv_heads;
     if (pt == 0) {
       if (a.q_tma) tma_prefetch_desc(&a.tm_q);
-      if (a.kv_tma) {
+      if (!kRows && a.kv_tma) {
         tma_prefetch_desc(&a.tm_k);
         tma_prefetch_desc(&a.tm_v);
       }
@@ -193,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       const int j = k >> 1;
       const bool is_v = k & 1;
       const int pos0 = unit.kv_lo + j * kBlockN;
-      if (a.kv_tma) {
+      if (!kRows && a.kv_tma) {
         if (pt == 0) {
           if (k >= kSlots) mbar_wait(&sm.empty[slot], ((k >> 2) - 1) & 1, wc);
           mbar_arrive_expect_tx(&sm.full[slot], kBlockN * D * 2);
@@ -228,13 +231,31 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
           }
           named_bar_sync(1, kProdThreads);
         }
-        const __nv_bfloat16* base = is_v ? a.v : a.k;
-        const uint32_t dst = smem_u32(sm.kv[slot]);
-        for (int c = pt; c < kBlockN * kChunks; c += kProdThreads) {
-          const int r = c / kChunks, ch = c % kChunks;
-          const int src = sm.rowsrc[r];
-          const __nv_bfloat16* g = src >= 0 ? base + ((size_t)src * Hk + unit.kv_head) * D + ch * 8 : base;
-          cp_async_16(dst + tile_off(r, ch), g, src >= 0 ? 16u : 0u);
+        if (kRows) {
+          // thread pt copies 16-byte column ch of rows r0, r0 + kRowStep, ...:
+          // the source row is read once per row and the column offset is fixed.
+          const __nv_bfloat16* base = (is_v ? a.v : a.k) + unit.kv_head * D;
+          const uint32_t dst = smem_u32(sm.kv[slot]);
+          constexpr int kRowStep = kProdThreads / kChunks;
+          const int ch = pt % kChunks;
+          const uint32_t col_off = (uint32_t)((ch >> 3) * (kTileM * 128) + ((ch & 7) << 4));
+          const size_t row_stride = (size_t)Hk * D;
+          for (int r = pt / kChunks; r < kBlockN; r += kRowStep) {
+            const int src = sm.rowsrc[r];
+            const __nv_bfloat16* g = src >= 0 ? base + (size_t)src * row_stride + ch * 8 : a.k;
+            cp_async_16(dst + r * 128 + (col_off ^ ((r & 7) << 4)), g, src >= 0 ? 16u : 0u);
+          }
+        } else {
+          // (the page-gather instance never runs this; it is kept so that its
+          // register allocation matches the measured fast build)
+          const __nv_bfloat16* base = is_v ? a.v : a.k;
+          const uint32_t dst = smem_u32(sm.kv[slot]);
+          for (int c = pt; c < kBlockN * kChunks; c += kProdThreads) {
+            const int r = c / kChunks, ch = c % kChunks;
+            const int src = sm.rowsrc[r];
+            const __nv_bfloat16* g = src >= 0 ? base + ((size_t)src * Hk + unit.kv_head) * D + ch * 8 : base;
+            cp_async_16(dst + tile_off(r, ch), g, src >= 0 ? 16u : 0u);
+          }
         }
         cp_async_arrive_noinc(&sm.full[slot]);
       }
@@ -243,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // Make sure no TMA write into this CTA's shared memory is still in flight at exit.
     if (pt == 0 && n_tiles > 0) {
       if (a.q_tma) mbar_drain(&sm.q_full, 0);
-      if (a.kv_tma)
+      if (!kRows && a.kv_tma)
         for (int k = 2 * n_tiles - 1; k >= 0 && k >= 2 * n_tiles - kSlots; --k)
           mbar_drain(&sm.full[k & (kSlots - 1)], (k >> 2) & 1);
     }
@@ -508,17 +529,23 @@ bool make_map(CUtensorMap* m, const void* base, int D, int heads, int64_t rows, 
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
-cudaError_t launch(const Args& a, cudaStream_t stream) {
+template <int D, bool kRows>
+cudaError_t launch_as(const Args& a, cudaStream_t stream) {
   const size_t smem = sizeof(Smem<D>) + 1024;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(prefill_kernel<D, kRows>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  prefill_kernel<D><<<a.g.num_units, kThreads, smem, stream>>>(a);
+  prefill_kernel<D, kRows><<<a.g.num_units, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch(const Args& a, cudaStream_t stream) {
+  return a.kv_tma ? launch_as<D, false>(a, stream) : launch_as<D, true>(a, stream);
 }
 
 }  // namespace

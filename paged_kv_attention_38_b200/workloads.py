@@ -254,15 +254,24 @@ SPARSE_DENSE_SWEEP = [(1, 512), (1, 2048), (1, 8192), (16, 512), (16, 2048), (16
 
 
 def sparse_vs_dense(batch: int, seq_len: int, contiguous: bool) -> PagedProblem:
-    """Causal prefill, 32 qo / 8 kv heads, head_dim 128, page_size 1. With
-    ``contiguous=False`` the token slots are scattered over the pool (vector sparse);
-    with ``contiguous=True`` the same tensors are laid out in order (dense ragged)."""
+    """Causal prefill, 32 qo / 8 kv heads, head_dim 128.
+
+    ``contiguous=False``: page_size 1 with the token slots scattered over the
+    pool (vector sparsity). ``contiguous=True``: the dense ragged layout of the
+    same problem, i.e. every request's K/V rows contiguous and in order; it is
+    described to the kernel as 64-slot pages with the identity page table,
+    which is the same memory layout ([total_kv, Hk, D] row-major) since every
+    length in the sweep is a multiple of 64."""
     seed = SEED_BASE + 3
     lens = [seq_len] * batch
-    kind = "dense" if contiguous else "sparse"
-    return make_problem(f"{kind}_prefill_causal_b{batch}_l{seq_len}_h32_kv8_d128_ps1", lens, lens,
+    if contiguous:
+        assert seq_len % 64 == 0
+        return make_problem(f"dense_prefill_causal_b{batch}_l{seq_len}_h32_kv8_d128", lens, lens,
+                            num_qo_heads=32, num_kv_heads=8, head_dim=128, page_size=64,
+                            causal=True, seed=seed, contiguous=True)
+    return make_problem(f"sparse_prefill_causal_b{batch}_l{seq_len}_h32_kv8_d128_ps1", lens, lens,
                         num_qo_heads=32, num_kv_heads=8, head_dim=128, page_size=1,
-                        causal=True, seed=seed, contiguous=contiguous)
+                        causal=True, seed=seed)
 
 
 def paged_decode(batch: int = 128, lo: int = 1024, hi: int = 8192) -> PagedProblem:

@@ -166,16 +166,17 @@ def test_sparse_vs_dense_sampled(bl):
                                                sp.kv_indices, sp.kv_last_page_len, 1, True, sp.sm_scale, b, pos)
         rows = [int(sp.qo_indptr[b]) + x for x in pos]
         assert_parity(o[rows], lse[rows], o_r, l_r, what=f"sparse {bl} req {b}")
-    # the dense (contiguous) layout of the same draw gives the same result
+    # the dense (contiguous) layout of the same keys and values gives the same result
     de = W.sparse_vs_dense(B, L, contiguous=True)
+    hk, d = sp.k_cache.shape[2], sp.k_cache.shape[3]
+    idx_s = torch.from_numpy(sp.kv_indices.astype(np.int64))
     k = torch.empty_like(de.k_cache)
     v = torch.empty_like(de.v_cache)
-    idx_s = torch.from_numpy(sp.kv_indices.astype(np.int64))
-    k[:len(idx_s)] = sp.k_cache[idx_s]
-    v[:len(idx_s)] = sp.v_cache[idx_s]
+    k.view(-1, hk, d)[:len(idx_s)] = sp.k_cache.view(-1, hk, d)[idx_s]
+    v.view(-1, hk, d)[:len(idx_s)] = sp.v_cache.view(-1, hk, d)[idx_s]
     de.k_cache, de.v_cache, de.q = k, v, sp.q
     o2, l2, _ = gpu_run(de)
-    assert torch.equal(o, o2) and torch.equal(lse, l2)
+    assert_parity(o2, l2, o.float().cpu().double().numpy(), lse.cpu().double().numpy(), what="dense vs sparse")
 
 
 # --------------------------------------------------------------------------- decode
