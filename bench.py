@@ -84,6 +84,45 @@ def decode_bytes(p: W.PagedProblem) -> float:
     return float(kv + q + o + lse + idx)
 
 
+# ----------------------------------------------------------------- profile figures
+
+PREFILL_SOURCES = ("prefill_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
+DECODE_SOURCES = ("decode_sm100.cu", "merge.cu", "sm100_ptx.cuh", "pkv_internal.h")
+MLA_SOURCES = ("mla_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
+
+
+def kernel_source_sha(files) -> str:
+    """Short hash of the CUDA sources a kernel is built from."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "paged_kv_attention_38_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def profiled_traffic(summary: str, files, kv_tokens=None):
+    """DRAM bytes per launch from a committed ncu summary under profiles/, or None
+    when the summary is missing or was taken on other kernel sources. A summary
+    taken on a smaller batch (it then records `kv_tokens`) is scaled to a launch
+    with `kv_tokens` keys, for kernels whose traffic is proportional to them."""
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.split(":", 1)[0] in ("source_sha", "dram_bytes_per_launch", "kv_tokens"):
+                k, v = line.split(":", 1)
+                fields[k] = v.strip()
+    if fields.get("source_sha") != kernel_source_sha(files) or "dram_bytes_per_launch" not in fields:
+        return None
+    traffic = float(fields["dram_bytes_per_launch"])
+    if "kv_tokens" in fields and kv_tokens is not None:
+        traffic *= kv_tokens / float(fields["kv_tokens"])
+    return traffic
+
+
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -378,13 +417,28 @@ def run_ours(args):
     peak_burst = float(peaks["bf16_tflops"])
     peak_sust = float(peaks.get("bf16_tflops_sustained", peak_burst))
     hbm = float(peaks["hbm_gbs"])
-    traffic = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tp):
-        with open(tp) as f:
-            tj = json.load(f)
-        if tj.get("kernel_version") == pkv.load_library().pkv_version().decode():
-            traffic = tj.get("prefill_bytes_per_launch")
+    roofs = {
+        "prefill_kernel<128> (h16/kv1/d128/ps64)": {
+            "bound": "tensor", "achieved": round(per_gpu_tflops, 2), "peak": peak_burst, "unit": "TFLOP/s",
+            "frac": round(per_gpu_tflops / peak_burst, 4), "frac_of_sustained": round(per_gpu_tflops / peak_sust, 4),
+            "traffic": profiled_traffic("prefill_gqa_h16_kv1_d128_ps64.md", PREFILL_SOURCES), "ms": round(pre_ms, 4)},
+        "decode_kernel<128> (b128/h32/kv8/d128/ps16)": {
+            "bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(dec_gbs / hbm, 4),
+            "traffic": profiled_traffic("decode_b32_h32_kv8_d128_ps16.md", DECODE_SOURCES,
+                                        kv_tokens=int(dec.p.kv_lens.sum())),
+            "ms": round(dec_ms, 4)},
+    }
+    if mla:
+        mla_tf = attention_flops(mla.p) / (mla_ms * 1e-3) / 1e12
+        roofs["mla_kernel (h16/ckv512/kpe64/ps1)"] = {
+            "bound": "tensor", "achieved": round(mla_tf, 2), "peak": peak_burst, "unit": "TFLOP/s",
+            "frac": round(mla_tf / peak_burst, 4),
+            "traffic": profiled_traffic("mla_h16_ckv512_kpe64_ps1.md", MLA_SOURCES), "ms": round(mla_ms, 4)}
+    dominant = max(roofs, key=lambda k: roofs[k]["ms"])
+    roofline = dict(roofs[dominant], kernel=dominant,
+                    peak_kind=f"{peak_kind} (burst bf16 for tensor-bound kernels timed alone between L2 flushes; "
+                              "copy bandwidth for HBM-bound)")
 
     if rank != 0:
         return
@@ -416,11 +470,8 @@ def run_ours(args):
                    "frac": round(dec_gbs / hbm, 4), "peak": hbm, "peak_kind": peak_kind,
                    "units": dec.plan.num_units, "merges": dec.plan.num_merges,
                    "workload": "paged_decode_b128_h32_kv8_d128_ps16, kv_len U[1024,8192]"},
-        "roofline": {"bound": "tensor", "achieved": round(per_gpu_tflops, 2), "peak": peak_burst,
-                     "unit": "TFLOP/s", "frac": round(per_gpu_tflops / peak_burst, 4),
-                     "frac_of_sustained": round(per_gpu_tflops / peak_sust, 4),
-                     "peak_kind": f"{peak_kind} burst bf16 (kernel timed alone between L2 flushes)",
-                     "traffic": traffic, "kernel": "prefill_kernel<128>"},
+        "roofline": roofline,
+        "rooflines": roofs,
         "e2e": {"value": round(pre_flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "includes": "plan + upload + H2D(q, k, v, kv_indices) + run + D2H(o, lse)"},
@@ -442,6 +493,7 @@ def run_ours(args):
 def run_only(args, device, flush):
     """One workload alone (for profiler captures): W warm-up and K timed launches."""
     makers = {"prefill": W.gqa_prefill, "decode": W.paged_decode, "mla": W.mla_prefill,
+              "decode_small": lambda: W.paged_decode(batch=32),
               "sparse": lambda: W.sparse_vs_dense(16, 2048, False),
               "dense": lambda: W.sparse_vs_dense(16, 2048, True)}
     c = Case(makers[args.only](), device)
@@ -451,7 +503,7 @@ def run_only(args, device, flush):
     f = attention_flops(c.p)
     print(json.dumps({"only": args.only, "ms_median": med, "ms_mean": mean,
                       "tflops": f / (med * 1e-3) / 1e12,
-                      "gbs": decode_bytes(c.p) / (med * 1e-3) / 1e9 if args.only == "decode" else None,
+                      "gbs": decode_bytes(c.p) / (med * 1e-3) / 1e9 if args.only.startswith("decode") else None,
                       "units": c.plan.num_units, "merges": c.plan.num_merges,
                       "clocks": sampler.summary()}), flush=True)
 
@@ -512,7 +564,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--sweep", action="store_true", help="also run the vector-sparse vs dense sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "mla", "sparse", "dense"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "decode_small", "mla", "sparse", "dense"], default=None,
                     help="time one workload alone (profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
