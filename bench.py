@@ -335,12 +335,29 @@ def dist_setup(n_gpus: int):
     return rank, world, local
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """The largest of every rank's `x` (all ranks call it, in the same order)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device="cuda") -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def job_throughput(local_work: float, local_ms: float, world: int, device="cuda"):
+    """Whole-job throughput of a weak-scaled run: the work every rank did, over
+    the slowest rank's time. Returns (work per second, max ms)."""
+    total = sum_over_ranks(local_work, world, device)
+    ms = max_over_ranks(local_ms, world, device)
+    return total / (ms * 1e-3), ms
 
 
 def barrier(world: int):
@@ -358,12 +375,13 @@ def run_ours(args):
 
     if args.only:
         return run_only(args, device, flush)
-    pre = Case(W.gqa_prefill(), device)
-    dec = Case(W.paged_decode(), device)
+    # one independent batch per rank (weak scaling: no data-path collective)
+    pre = Case(W.gqa_prefill(shard=rank), device)
+    dec = Case(W.paged_decode(shard=rank), device)
     cases = [pre, dec]
     mla = None
     try:
-        mla = Case(W.mla_prefill(), device)
+        mla = Case(W.mla_prefill(shard=rank), device)
         mla.run()
         torch.cuda.synchronize()
         cases.append(mla)
@@ -399,20 +417,19 @@ def run_ours(args):
     def mean_ms(c):
         return float(np.mean([a.elapsed_time(b) for a, b in ev[id(c)]]))
 
-    pre_ms = max_over_ranks(mean_ms(pre), world)
-    dec_ms = max_over_ranks(mean_ms(dec), world)
-    mla_ms = max_over_ranks(mean_ms(mla), world) if mla else None
-    step_ms = pre_ms + dec_ms + (mla_ms or 0.0)
-
     pre_flops = attention_flops(pre.p)
     dec_bytes = decode_bytes(dec.p)
-    tflops = pre_flops * world / (pre_ms * 1e-3) / 1e12
+    job_flops_s, pre_ms = job_throughput(pre_flops, mean_ms(pre), world)
+    job_bytes_s, dec_ms = job_throughput(dec_bytes, mean_ms(dec), world)
+    mla_ms = max_over_ranks(mean_ms(mla), world) if mla else None
+    step_ms = pre_ms + dec_ms + (mla_ms or 0.0)
+    tflops = job_flops_s / 1e12
     per_gpu_tflops = pre_flops / (pre_ms * 1e-3) / 1e12
     dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
 
     # e2e through the public API with host buffers
-    e2e_ms, h2d, d2h = e2e_prefill(pre.p, device, max(2, min(args.steps, 10)), 2)
-    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e_local_ms, h2d, d2h = e2e_prefill(pre.p, device, max(2, min(args.steps, 10)), 2)
+    e2e_flops_s, e2e_ms = job_throughput(pre_flops, e2e_local_ms, world)
 
     peak_burst = float(peaks["bf16_tflops"])
     peak_sust = float(peaks.get("bf16_tflops_sustained", peak_burst))
@@ -466,13 +483,13 @@ def run_ours(args):
         "pct_bf16_peak": round(100 * per_gpu_tflops / peak_burst, 2),
         "prefill": {"ms": round(pre_ms, 4), "flops": pre_flops, "tflops_per_gpu": round(per_gpu_tflops, 2),
                     "units": pre.plan.num_units, "merges": pre.plan.num_merges},
-        "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "ms": round(dec_ms, 4), "bytes": dec_bytes,
+        "decode": {"value": round(dec_gbs, 1), "job_value": round(job_bytes_s / 1e9, 1), "unit": "GB/s", "ms": round(dec_ms, 4), "bytes": dec_bytes,
                    "frac": round(dec_gbs / hbm, 4), "peak": hbm, "peak_kind": peak_kind,
                    "units": dec.plan.num_units, "merges": dec.plan.num_merges,
                    "workload": "paged_decode_b128_h32_kv8_d128_ps16, kv_len U[1024,8192]"},
         "roofline": roofline,
         "rooflines": roofs,
-        "e2e": {"value": round(pre_flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(e2e_flops_s / 1e12, 2), "unit": "TFLOP/s",
                 "ms": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "includes": "plan + upload + H2D(q, k, v, kv_indices) + run + D2H(o, lse)"},
         "gpu_launches": int(args.steps * sum(c.launches for c in cases)),

@@ -151,16 +151,6 @@ def _valid_slot_mask(kv_indptr, kv_indices, last, page_size, pool_pages) -> torc
     return valid
 
 
-def _pools(shape_k, shape_v, valid, gen):
-    """Pools whose valid slots hold N(0,1) bf16 and whose other slots hold the sentinel."""
-    k = _randn_bf16(shape_k, gen)
-    v = _randn_bf16(shape_v, gen)
-    inv = ~valid
-    k[inv] = SENTINEL_K
-    v[inv] = SENTINEL_V
-    return k, v
-
-
 def make_problem(name: str, qo_lens, kv_lens, *, num_qo_heads: int, num_kv_heads: int,
                  head_dim: int, page_size: int, causal: bool, seed: int,
                  head_dim_v: Optional[int] = None, sm_scale: Optional[float] = None,
@@ -239,10 +229,11 @@ def tiny_prefill() -> PagedProblem:
                         causal=True, seed=SEED_BASE + 1, pool_pages=16)
 
 
-def gqa_prefill(batch: int = 8, lo: int = 512, hi: int = 4096) -> PagedProblem:
+def gqa_prefill(batch: int = 8, lo: int = 512, hi: int = 4096, shard: int = 0) -> PagedProblem:
     """Causal GQA paged prefill: qo_len = kv_len ~ U[512, 4096], 16 qo / 1 kv head,
-    head_dim 128, page_size 64, permuted pool (h16/kv1/d128/ps64)."""
-    seed = SEED_BASE + 2
+    head_dim 128, page_size 64, permuted pool (h16/kv1/d128/ps64). `shard` draws
+    another independent batch of the same shape (one per data-parallel rank)."""
+    seed = SEED_BASE + 2 + 10000 * shard
     lens = uniform_lengths(batch, lo, hi, _gen(seed + 7))
     return make_problem("gqa_paged_prefill_causal_h16_kv1_d128_ps64", lens, lens,
                         num_qo_heads=16, num_kv_heads=1, head_dim=128, page_size=64,
@@ -274,37 +265,20 @@ def sparse_vs_dense(batch: int, seq_len: int, contiguous: bool) -> PagedProblem:
                         causal=True, seed=seed)
 
 
-def paged_decode(batch: int = 128, lo: int = 1024, hi: int = 8192) -> PagedProblem:
+def paged_decode(batch: int = 128, lo: int = 1024, hi: int = 8192, shard: int = 0) -> PagedProblem:
     """Paged decode: q_len 1, 32 qo / 8 kv heads, head_dim 128, page_size 16,
     kv_len ~ U[1024, 8192]. Non-causal (one query sees every key)."""
-    seed = SEED_BASE + 4
+    seed = SEED_BASE + 4 + 10000 * shard
     kv = uniform_lengths(batch, lo, hi, _gen(seed + 7))
     return make_problem("paged_decode_b128_h32_kv8_d128_ps16", [1] * batch, kv,
                         num_qo_heads=32, num_kv_heads=8, head_dim=128, page_size=16,
                         causal=False, seed=seed)
 
 
-def mla_prefill(batch: int = 4, lo: int = 256, hi: int = 2048) -> PagedProblem:
+def mla_prefill(batch: int = 4, lo: int = 256, hi: int = 2048, shard: int = 0) -> PagedProblem:
     """Absorbed MLA causal paged prefill, 16 heads, ckv 512 + kpe 64, page_size 1,
     sm_scale 1/sqrt(192) (h16/ckv512/kpe64/ps1)."""
-    seed = SEED_BASE + 5
+    seed = SEED_BASE + 5 + 10000 * shard
     lens = uniform_lengths(batch, lo, hi, _gen(seed + 7))
     return make_mla_problem("mla_paged_prefill_causal_h16_ckv512_kpe64_ps1", lens, lens,
                             num_heads=16, seed=seed)
-
-
-def causal_flops(p: PagedProblem) -> float:
-    """Algorithmic FLOPs of a causal (or full) attention pass: only visible (query, key)
-    pairs count, 2 FLOPs per multiply-add, for QK^T (width head_dim [+ pe]) and PV."""
-    qo, kv = p.qo_lens, p.kv_lens
-    pairs = 0
-    for a, b in zip(qo.tolist(), kv.tolist()):
-        if p.causal:
-            # query i sees keys j <= i + (b - a); count them for i in [0, a)
-            d = b - a
-            lo_vis = np.clip(np.arange(a) + d + 1, 0, b)
-            pairs += int(lo_vis.sum())
-        else:
-            pairs += a * b
-    width = p.head_dim + p.head_dim_pe + p.head_dim_v
-    return 2.0 * width * p.num_qo_heads * pairs
