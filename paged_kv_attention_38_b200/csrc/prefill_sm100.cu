@@ -270,7 +270,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     }
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
-    if (lane == 0 && n_tiles > 0) {
+    // The whole warp runs this loop (waits, descriptor arithmetic) so its
+    // operands stay in uniform registers; one elected lane issues each
+    // tcgen05.mma / commit. (Run from a single divergent lane, the same loop
+    // cost about twice the instructions per MMA and left the tensor core idle.)
+    if (n_tiles > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kTileM, kBlockN, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kTileM, D, true);
       auto wait_item = [&](int k) {
@@ -278,40 +282,37 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         fence_proxy_async_smem();  // cp.async rows were written through the generic proxy
         tc_fence_after();
       };
-      // Descriptors are built once; a K-step only moves the start address,
-      // which is the low 14-bit field (addr >> 4), so it is added in place.
-      uint64_t dq[kTiles], dk[kSlots], dv[kSlots];
-#pragma unroll
-      for (int i = 0; i < kTiles; ++i) dq[i] = sdesc_sw128(smem_u32(sm.q[i]), 16, 1024);
-#pragma unroll
-      for (int sl = 0; sl < kSlots; ++sl) {
-        dk[sl] = sdesc_sw128(smem_u32(sm.kv[sl]), 16, 1024);
-        dv[sl] = sdesc_sw128(smem_u32(sm.kv[sl]), kBlockN * 128, 1024);
-      }
+      // Descriptors are built once; a K-step or another buffer only moves the
+      // start address, the low 14-bit field (addr >> 4), so offsets are added in place.
+      const uint64_t dq0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(sm.kv[0]), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(sm.kv[0]), kBlockN * 128, 1024);
+      constexpr uint32_t kQStep = (kTileM * D * 2) >> 4;      // one Q tile
+      constexpr uint32_t kSlotStep = (kBlockN * D * 2) >> 4;  // one K/V slot
       auto issue_s = [&](int i, int j) {
-        const uint64_t bq = dq[i], bk = dk[(2 * j) & (kSlots - 1)];
+        const uint64_t bq = dq0 + i * kQStep, bk = dk0 + ((2 * j) & (kSlots - 1)) * kSlotStep;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
-          umma_bf16(tmem + i * kBlockN, bq + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ss_elect(tmem + i * kBlockN, bq + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
         }
       };
       // O_i += P_i V_j for kv columns [64h, 64h + 64) of this tile: K-steps 4h..4h+3.
       auto issue_pv_half = [&](int i, int j, int h) {
-        const uint64_t bv = dv[(2 * j + 1) & (kSlots - 1)];
+        const uint64_t bv = dv0 + ((2 * j + 1) & (kSlots - 1)) * kSlotStep;
 #pragma unroll
         for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
-          umma_bf16_ts(tmem + 256 + i * 128, tmem + i * kBlockN + kk * 8, bv + ((kk * 16 * 128) >> 4), idesc_o,
-                       (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts_elect(tmem + 256 + i * 128, tmem + i * kBlockN + kk * 8, bv + ((kk * 16 * 128) >> 4),
+                             idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
       };
       mbar_wait(&sm.q_full, 0, wc);
       fence_proxy_async_smem();
       wait_item(0);
       issue_s(0, 0);
-      umma_commit(&sm.s_full[0]);
+      umma_commit_elect(&sm.s_full[0]);
       issue_s(1, 0);
-      umma_commit(&sm.s_full[1]);
-      umma_commit(&sm.empty[0]);
+      umma_commit_elect(&sm.s_full[1]);
+      umma_commit_elect(&sm.empty[0]);
       for (int j = 0; j < n_tiles; ++j) {
         const bool more = j + 1 < n_tiles;
         mbar_wait(&sm.p_half[0][0], j & 1, wc);
@@ -323,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         if (more) {
           wait_item(2 * j + 2);
           issue_s(0, j + 1);
-          umma_commit(&sm.s_full[0]);
+          umma_commit_elect(&sm.s_full[0]);
         }
         mbar_wait(&sm.p_half[1][0], j & 1, wc);
         tc_fence_after();
@@ -331,14 +332,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         mbar_wait(&sm.p_half[1][1], j & 1, wc);
         tc_fence_after();
         issue_pv_half(1, j, 1);
-        umma_commit(&sm.empty[(2 * j + 1) & (kSlots - 1)]);
+        umma_commit_elect(&sm.empty[(2 * j + 1) & (kSlots - 1)]);
         if (more) {
           issue_s(1, j + 1);
-          umma_commit(&sm.s_full[1]);
-          umma_commit(&sm.empty[(2 * j + 2) & (kSlots - 1)]);
+          umma_commit_elect(&sm.s_full[1]);
+          umma_commit_elect(&sm.empty[(2 * j + 2) & (kSlots - 1)]);
         }
       }
-      umma_commit(&sm.o_final);
+      umma_commit_elect(&sm.o_final);
       mbar_drain(&sm.o_final, 0);  // no MMA may still run when TMEM is released
     }
     __syncwarp();
