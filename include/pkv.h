@@ -181,7 +181,9 @@ PKV_API pkv_status pkv_device_status(const pkv_plan* plan, void* stream, int32_t
 
 /* Introspection (host only, no device access):
  *   key 0 kernel kind (0 prefill, 1 decode, 2 MLA), 1 work units, 2 merge tasks,
- *   3 partial slots, 4 rows per partial slot, 5 SMs planned for, 6 KV chunk. */
+ *   3 partial slots, 4 rows per partial slot, 5 SMs planned for, 6 KV chunk,
+ *   7 CTAs of the main launch (prefill: persistent CTAs, each running a fixed
+ *   list of work units; decode / MLA: one CTA per work unit). */
 PKV_API int64_t pkv_plan_info(const pkv_plan* plan, int32_t key);
 
 /* Copy the work list (8 int32 per unit: req, kv_head, row0, rows, kv_lo, kv_hi,
@@ -190,6 +192,12 @@ PKV_API int32_t pkv_plan_work_units(const pkv_plan* plan, int32_t* out, int32_t 
 
 /* Copy the merge list (8 int32 per task: req, kv_head, row0, rows, slot0, num, 0, 0). */
 PKV_API int32_t pkv_plan_merge_tasks(const pkv_plan* plan, int32_t* out, int32_t capacity);
+
+/* Copy the persistent-CTA schedule of a prefill plan: num_ctas + 1 offsets
+ * into the work list (CTA b runs units [out[b], out[b + 1]) in order) into
+ * `out` (HOST, capacity in int32). Returns the entries copied; 0 for decode and
+ * MLA plans, whose CTAs each run one unit. */
+PKV_API int32_t pkv_plan_cta_units(const pkv_plan* plan, int32_t* out, int32_t capacity);
 
 PKV_API void pkv_plan_destroy(pkv_plan* plan);
 

@@ -67,6 +67,7 @@ _SIGS = {
     "pkv_plan_info": (ctypes.c_int64, [_P, ctypes.c_int32]),
     "pkv_plan_work_units": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
     "pkv_plan_merge_tasks": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
+    "pkv_plan_cta_units": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
     "pkv_plan_destroy": (None, [_P]),
     "pkv_last_error": (ctypes.c_char_p, []),
     "pkv_version": (ctypes.c_char_p, []),
@@ -147,6 +148,10 @@ class Plan:
         return self.info(6)
 
     @property
+    def num_ctas(self) -> int:
+        return self.info(7)
+
+    @property
     def workspace_bytes(self) -> int:
         return int(load_library().pkv_plan_workspace_bytes(self._h))
 
@@ -160,6 +165,13 @@ class Plan:
         n = self.num_merges
         out = np.zeros((max(n, 1), 8), dtype=np.int32)
         got = load_library().pkv_plan_merge_tasks(self._h, _i32p(out), n)
+        return out[:got]
+
+    def cta_units(self) -> np.ndarray:
+        """Persistent prefill schedule: CTA b runs work units [out[b], out[b+1]); empty otherwise."""
+        n = self.num_ctas + 1
+        out = np.zeros(n, dtype=np.int32)
+        got = load_library().pkv_plan_cta_units(self._h, _i32p(out), n)
         return out[:got]
 
     def upload(self, device=None, stream=None):

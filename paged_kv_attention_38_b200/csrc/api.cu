@@ -30,9 +30,9 @@ struct pkv_plan {
   Schedule sched;
   const int32_t* kv_indices = nullptr;  // device, borrowed
   // workspace layout (byte offsets)
-  size_t off_status = 0, off_units = 0, off_merges = 0, off_reqs = 0, off_lse = 0, off_o = 0, total = 0;
+  size_t off_status = 0, off_units = 0, off_merges = 0, off_reqs = 0, off_cta = 0, off_lse = 0, off_o = 0, total = 0;
   size_t staging_bytes = 0;
-  void* staging = nullptr;  // host copy of [status | units | merges | reqs]
+  void* staging = nullptr;  // host copy of [status | units | merges | reqs | cta_ptr]
   bool staging_pinned = false;
   DeviceView dv{};
   bool uploaded = false;
@@ -69,6 +69,8 @@ void layout_workspace(pkv_plan* p) {
   off = align256(off + s.merges.size() * sizeof(MergeTask));
   p->off_reqs = off;
   off = align256(off + s.reqs.size() * sizeof(ReqInfo));
+  p->off_cta = off;
+  off = align256(off + s.cta_ptr.size() * sizeof(int32_t));
   p->staging_bytes = off;
   p->off_lse = off;
   off = align256(off + (size_t)s.num_slots * s.geom.part_rows * sizeof(float));
@@ -169,6 +171,7 @@ pkv_status pkv_plan_upload(pkv_plan* p, void* workspace, size_t bytes, void* str
     if (!s.units.empty()) std::memcpy(h + p->off_units, s.units.data(), s.units.size() * sizeof(WorkUnit));
     if (!s.merges.empty()) std::memcpy(h + p->off_merges, s.merges.data(), s.merges.size() * sizeof(MergeTask));
     if (!s.reqs.empty()) std::memcpy(h + p->off_reqs, s.reqs.data(), s.reqs.size() * sizeof(ReqInfo));
+    if (!s.cta_ptr.empty()) std::memcpy(h + p->off_cta, s.cta_ptr.data(), s.cta_ptr.size() * sizeof(int32_t));
   }
   uint8_t* d = static_cast<uint8_t*>(workspace);
   cudaError_t e = cudaMemcpyAsync(d, p->staging, p->staging_bytes, cudaMemcpyHostToDevice,
@@ -180,6 +183,7 @@ pkv_status pkv_plan_upload(pkv_plan* p, void* workspace, size_t bytes, void* str
   p->dv.part_lse = reinterpret_cast<float*>(d + p->off_lse);
   p->dv.part_o = reinterpret_cast<float*>(d + p->off_o);
   p->dv.status = reinterpret_cast<int*>(d + p->off_status);
+  p->dv.cta_ptr = reinterpret_cast<const int32_t*>(d + p->off_cta);
   p->uploaded = true;
   return PKV_OK;
 }
@@ -266,6 +270,7 @@ int64_t pkv_plan_info(const pkv_plan* p, int32_t key) {
     case 4: return s.geom.part_rows;
     case 5: return s.num_sms;
     case 6: return s.kv_chunk;
+    case 7: return s.geom.num_ctas;
     default: return -1;
   }
 }
@@ -281,6 +286,13 @@ int32_t pkv_plan_merge_tasks(const pkv_plan* p, int32_t* out, int32_t capacity) 
   if (!p || !out || capacity <= 0) return 0;
   const int32_t n = (int32_t)std::min<size_t>(p->sched.merges.size(), (size_t)capacity);
   std::memcpy(out, p->sched.merges.data(), (size_t)n * sizeof(MergeTask));
+  return n;
+}
+
+int32_t pkv_plan_cta_units(const pkv_plan* p, int32_t* out, int32_t capacity) {
+  if (!p || !out || capacity <= 0) return 0;
+  const int32_t n = (int32_t)std::min<size_t>(p->sched.cta_ptr.size(), (size_t)capacity);
+  if (n > 0) std::memcpy(out, p->sched.cta_ptr.data(), (size_t)n * sizeof(int32_t));
   return n;
 }
 

@@ -71,6 +71,7 @@ struct LaunchGeom {
   int32_t num_units;
   int32_t num_merge;
   int32_t total_q;        // rows of q (tokens)
+  int32_t num_ctas;       // CTAs of the main launch (prefill: persistent, one unit list each)
 };
 
 // Device pointers into the workspace after upload.
@@ -81,6 +82,7 @@ struct DeviceView {
   float* part_o;          // [num_slots, part_rows, head_dim_v]
   float* part_lse;        // [num_slots, part_rows]
   int* status;            // device status word (0 = ok)
+  const int32_t* cta_ptr; // prefill: CTA b runs units [cta_ptr[b], cta_ptr[b + 1])
 };
 
 }  // namespace pkv

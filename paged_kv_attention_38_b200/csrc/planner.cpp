@@ -12,7 +12,10 @@
 
 #include <algorithm>
 #include <cmath>
+#include <functional>
 #include <numeric>
+#include <queue>
+#include <utility>
 
 namespace pkv {
 
@@ -161,6 +164,32 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
     return (a.kv_hi - a.kv_lo) > (b.kv_hi - b.kv_lo);
   });
 
+  // Prefill runs persistent CTAs (one per SM), each over a fixed list of
+  // units. Greedy list scheduling in the longest-first order above: each unit
+  // goes to the CTA with the least work so far, counted in KV tiles plus one
+  // tile for the unit's own start and end. The units are then stored CTA by CTA.
+  int32_t num_ctas = (int32_t)s.units.size();
+  if (s.kind == kKindPrefill && !s.units.empty()) {
+    num_ctas = (int32_t)std::min<size_t>((size_t)num_sms, s.units.size());
+    using Load = std::pair<int64_t, int32_t>;  // (work so far, cta)
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int32_t c = 0; c < num_ctas; ++c) heap.push({0, c});
+    std::vector<std::vector<WorkUnit>> lists((size_t)num_ctas);
+    for (const WorkUnit& u : s.units) {
+      Load top = heap.top();
+      heap.pop();
+      lists[(size_t)top.second].push_back(u);
+      top.first += (u.kv_hi - u.kv_lo + kBlockN - 1) / kBlockN + 1;
+      heap.push(top);
+    }
+    s.units.clear();
+    s.cta_ptr.assign(1, 0);
+    for (const auto& l : lists) {
+      s.units.insert(s.units.end(), l.begin(), l.end());
+      s.cta_ptr.push_back((int32_t)s.units.size());
+    }
+  }
+
   LaunchGeom& gm = s.geom;
   gm.num_qo_heads = in.num_qo_heads;
   gm.num_kv_heads = in.num_kv_heads;
@@ -176,6 +205,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   gm.num_units = (int32_t)s.units.size();
   gm.num_merge = (int32_t)s.merges.size();
   gm.total_q = in.batch > 0 ? in.qo_indptr[in.batch] : 0;
+  gm.num_ctas = num_ctas;
   *out = std::move(s);
   return 0;
 }

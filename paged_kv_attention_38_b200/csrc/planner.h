@@ -40,6 +40,7 @@ struct Schedule {
   std::vector<ReqInfo> reqs;
   std::vector<WorkUnit> units;
   std::vector<MergeTask> merges;
+  std::vector<int32_t> cta_ptr;  // prefill: [num_ctas + 1] offsets of each CTA's units
   int32_t num_slots = 0;
   int32_t kv_chunk = 0;   // chunk used (0 = no split)
   int32_t num_sms = 0;

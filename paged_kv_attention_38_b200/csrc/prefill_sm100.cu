@@ -77,11 +77,13 @@ struct __align__(1024) Smem {
   __nv_bfloat16 q[kTiles][kTileM * D];
   __nv_bfloat16 kv[kSlots][kBlockN * D];
   uint64_t q_full;
+  uint64_t q_empty;  // the unit's last QK^T MMAs are done: Q may be overwritten
   uint64_t full[kSlots];
   uint64_t empty[kSlots];
   uint64_t s_full[kTiles];
   uint64_t p_half[kTiles][2];  // P_i columns [0,64) / [64,128) written
-  uint64_t o_final;
+  uint64_t o_final[kTiles];    // O_i of the unit is complete
+  uint64_t mma_done;           // every MMA of the CTA is complete (exit)
   int32_t rowsrc[kBlockN];  // cp.async gather: pool row of each tile row, -1 = zero fill
   uint32_t tmem_base;
   int abort_flag;
@@ -107,6 +109,12 @@ struct Args {
 // kRows: K/V arrive as single rows by cp.async (page_size < 8) instead of whole
 // pages by TMA. A template parameter, so each instance holds only its own
 // producer code (the instances' register allocation is then independent).
+//
+// Persistent: CTA b runs work units [cta_ptr[b], cta_ptr[b + 1]) back to back.
+// Barrier phases run on across units (counters of K/V items, KV tiles and
+// units with keys), so the producer streams the next unit's Q and K/V and the
+// tensor core starts its first QK^T while the softmax warps still write the
+// previous unit's output.
 template <int D, bool kRows>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Args a) {
   extern __shared__ uint8_t smem_raw[];
@@ -114,14 +122,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-
-  const WorkUnit unit = a.dv.units[blockIdx.x];
-  const ReqInfo req = a.dv.reqs[unit.req];
+  const int u_begin = a.dv.cta_ptr[blockIdx.x];
+  const int u_end = a.dv.cta_ptr[blockIdx.x + 1];
   const int G = a.g.group;
-  const int n_tiles = (unit.kv_hi - unit.kv_lo + kBlockN - 1) / kBlockN;
+  auto tiles_of = [](const WorkUnit& u) { return (u.kv_hi - u.kv_lo + kBlockN - 1) / kBlockN; };
 
   if (tid == 0) {
     mbar_init(&sm.q_full, a.q_tma ? 1 : kProdThreads);
+    mbar_init(&sm.q_empty, 1);
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&sm.full[s], (!kRows && a.kv_tma) ? 1 : kProdThreads);
       mbar_init(&sm.empty[s], 1);
@@ -130,8 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.p_half[i][0], kTileM);
       mbar_init(&sm.p_half[i][1], kTileM);
+      mbar_init(&sm.o_final[i], 1);
     }
-    mbar_init(&sm.o_final, 1);
+    mbar_init(&sm.mma_done, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -162,111 +171,131 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         tma_prefetch_desc(&a.tm_v);
       }
     }
-    // ---- Q tiles (nothing to load when the unit has no key: the CTA only writes zeros)
-    if (n_tiles == 0) {
-    } else if (a.q_tma) {
-      if (pt == 0) {
-        mbar_arrive_expect_tx(&sm.q_full, kTiles * kTileM * D * 2);
-        for (int i = 0; i < kTiles; ++i) {
-          const int t0 = (unit.row0 + i * kTileM) / G;
-#pragma unroll
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(smem_u32(sm.q[i]) + h * (kTileM * 128), &a.tm_q, &sm.q_full, h * 64, unit.kv_head * G,
-                        req.q_start + t0);
-        }
-      }
-    } else {
-      const size_t head_stride = (size_t)a.g.num_qo_heads * D;
-      for (int c = pt; c < kTiles * kTileM * kChunks; c += kProdThreads) {
-        const int r = c / kChunks, ch = c % kChunks;
-        const bool ok = r < unit.rows;
-        const __nv_bfloat16* src = a.q;
-        if (ok) {
-          const int pr = unit.row0 + r;
-          src = a.q + (size_t)(req.q_start + pr / G) * head_stride + (size_t)(unit.kv_head * G + pr % G) * D + ch * 8;
-        }
-        cp_async_16(smem_u32(sm.q[r / kTileM]) + tile_off(r % kTileM, ch), src, ok ? 16u : 0u);
-      }
-      cp_async_arrive_noinc(&sm.q_full);
-    }
-    // ---- K / V items: item 2j is K_j, item 2j+1 is V_j, slot = item % kSlots
-    const int n_pages_req = (req.kv_len + P - 1) >> shift;
-    for (int k = 0; k < 2 * n_tiles; ++k) {
-      const int slot = k & (kSlots - 1);
-      const int j = k >> 1;
-      const bool is_v = k & 1;
-      const int pos0 = unit.kv_lo + j * kBlockN;
-      if (!kRows && a.kv_tma) {
+    // Q tile i of a unit by TMA: rows of 128 / G tokens x G heads from this token on.
+    auto q_token = [&](const WorkUnit& u, const ReqInfo& rq, int i) { return rq.q_start + (u.row0 + i * kTileM) / G; };
+    int kc = 0;  // K/V items issued (item 2j is K_j, 2j+1 is V_j; slot = item % kSlots)
+    int uq = 0;  // units with keys whose Q was loaded
+    for (int ui = u_begin; ui < u_end; ++ui) {
+      const WorkUnit unit = a.dv.units[ui];
+      const int n_tiles = tiles_of(unit);
+      if (n_tiles == 0) continue;  // the CTA only writes zeros for it
+      const ReqInfo req = a.dv.reqs[unit.req];
+      // ---- Q tiles, once the previous unit's QK^T MMAs have read the old ones
+      if (uq > 0) mbar_wait(&sm.q_empty, (uq - 1) & 1, wc);
+      if (a.q_tma) {
         if (pt == 0) {
-          if (k >= kSlots) mbar_wait(&sm.empty[slot], ((k >> 2) - 1) & 1, wc);
-          mbar_arrive_expect_tx(&sm.full[slot], kBlockN * D * 2);
-          const CUtensorMap* tm = is_v ? &a.tm_v : &a.tm_k;
-          const uint32_t dst = smem_u32(sm.kv[slot]);
-          if (P >= kBlockN) {
-            const int page = __ldg(a.kv_indices + req.page0 + (pos0 >> shift));
-            const int row = page * P + (pos0 & (P - 1));
+          mbar_arrive_expect_tx(&sm.q_full, kTiles * kTileM * D * 2);
+          for (int i = 0; i < kTiles; ++i) {
+            const int tok = q_token(unit, req, i);
 #pragma unroll
-            for (int h = 0; h < D / 64; ++h) tma_load_3d(dst + h * (kTileM * 128), tm, &sm.full[slot], h * 64, unit.kv_head, row);
-          } else {
-            const int npc = kBlockN >> shift;
-            const int lp0 = pos0 >> shift;
-            for (int pi = 0; pi < npc; ++pi) {
-              const int lp = lp0 + pi;
-              const int row = lp < n_pages_req ? __ldg(a.kv_indices + req.page0 + lp) * P : a.oob_row;
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d(smem_u32(sm.q[i]) + h * (kTileM * 128), &a.tm_q, &sm.q_full, h * 64, unit.kv_head * G, tok);
+          }
+          // warm L2 with the next unit's Q so its load at the unit boundary is short
+          if (ui + 1 < u_end) {
+            const WorkUnit nu = a.dv.units[ui + 1];
+            const ReqInfo nr = a.dv.reqs[nu.req];
+            for (int i = 0; i < kTiles; ++i)
 #pragma unroll
               for (int h = 0; h < D / 64; ++h)
-                tma_load_3d(dst + h * (kTileM * 128) + pi * P * 128, tm, &sm.full[slot], h * 64, unit.kv_head, row);
-            }
+                tma_prefetch_l2_3d(&a.tm_q, h * 64, nu.kv_head * G, q_token(nu, nr, i));
           }
         }
       } else {
-        if (k >= kSlots) mbar_wait(&sm.empty[slot], ((k >> 2) - 1) & 1, wc);
-        if (!is_v) {
-          named_bar_sync(1, kProdThreads);  // the previous tile's copies have all been issued
-          for (int r = pt; r < kBlockN; r += kProdThreads) {
-            const int pos = pos0 + r;
-            int src = -1;
-            if (pos < unit.kv_hi) src = __ldg(a.kv_indices + req.page0 + (pos >> shift)) * P + (pos & (P - 1));
-            sm.rowsrc[r] = src;
+        const size_t head_stride = (size_t)a.g.num_qo_heads * D;
+        for (int c = pt; c < kTiles * kTileM * kChunks; c += kProdThreads) {
+          const int r = c / kChunks, ch = c % kChunks;
+          const bool ok = r < unit.rows;
+          const __nv_bfloat16* src = a.q;
+          if (ok) {
+            const int pr = unit.row0 + r;
+            src = a.q + (size_t)(req.q_start + pr / G) * head_stride + (size_t)(unit.kv_head * G + pr % G) * D + ch * 8;
           }
-          named_bar_sync(1, kProdThreads);
+          cp_async_16(smem_u32(sm.q[r / kTileM]) + tile_off(r % kTileM, ch), src, ok ? 16u : 0u);
         }
-        if (kRows) {
-          // thread pt copies 16-byte column ch of rows r0, r0 + kRowStep, ...:
-          // the source row is read once per row and the column offset is fixed.
-          const __nv_bfloat16* base = (is_v ? a.v : a.k) + unit.kv_head * D;
-          const uint32_t dst = smem_u32(sm.kv[slot]);
-          constexpr int kRowStep = kProdThreads / kChunks;
-          const int ch = pt % kChunks;
-          const uint32_t col_off = (uint32_t)((ch >> 3) * (kTileM * 128) + ((ch & 7) << 4));
-          const size_t row_stride = (size_t)Hk * D;
-          for (int r = pt / kChunks; r < kBlockN; r += kRowStep) {
-            const int src = sm.rowsrc[r];
-            const __nv_bfloat16* g = src >= 0 ? base + (size_t)src * row_stride + ch * 8 : a.k;
-            cp_async_16(dst + r * 128 + (col_off ^ ((r & 7) << 4)), g, src >= 0 ? 16u : 0u);
+        cp_async_arrive_noinc(&sm.q_full);
+      }
+      ++uq;
+      // ---- K / V items
+      const int n_pages_req = (req.kv_len + P - 1) >> shift;
+      for (int k = 0; k < 2 * n_tiles; ++k, ++kc) {
+        const int slot = kc & (kSlots - 1);
+        const int j = k >> 1;
+        const bool is_v = k & 1;
+        const int pos0 = unit.kv_lo + j * kBlockN;
+        if (!kRows && a.kv_tma) {
+          if (pt == 0) {
+            if (kc >= kSlots) mbar_wait(&sm.empty[slot], ((kc >> 2) - 1) & 1, wc);
+            mbar_arrive_expect_tx(&sm.full[slot], kBlockN * D * 2);
+            const CUtensorMap* tm = is_v ? &a.tm_v : &a.tm_k;
+            const uint32_t dst = smem_u32(sm.kv[slot]);
+            if (P >= kBlockN) {
+              const int page = __ldg(a.kv_indices + req.page0 + (pos0 >> shift));
+              const int row = page * P + (pos0 & (P - 1));
+#pragma unroll
+              for (int h = 0; h < D / 64; ++h) tma_load_3d(dst + h * (kTileM * 128), tm, &sm.full[slot], h * 64, unit.kv_head, row);
+            } else {
+              const int npc = kBlockN >> shift;
+              const int lp0 = pos0 >> shift;
+              for (int pi = 0; pi < npc; ++pi) {
+                const int lp = lp0 + pi;
+                const int row = lp < n_pages_req ? __ldg(a.kv_indices + req.page0 + lp) * P : a.oob_row;
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h)
+                  tma_load_3d(dst + h * (kTileM * 128) + pi * P * 128, tm, &sm.full[slot], h * 64, unit.kv_head, row);
+              }
+            }
           }
         } else {
-          // (the page-gather instance never runs this; it is kept so that its
-          // register allocation matches the measured fast build)
-          const __nv_bfloat16* base = is_v ? a.v : a.k;
-          const uint32_t dst = smem_u32(sm.kv[slot]);
-          for (int c = pt; c < kBlockN * kChunks; c += kProdThreads) {
-            const int r = c / kChunks, ch = c % kChunks;
-            const int src = sm.rowsrc[r];
-            const __nv_bfloat16* g = src >= 0 ? base + ((size_t)src * Hk + unit.kv_head) * D + ch * 8 : base;
-            cp_async_16(dst + tile_off(r, ch), g, src >= 0 ? 16u : 0u);
+          if (kc >= kSlots) mbar_wait(&sm.empty[slot], ((kc >> 2) - 1) & 1, wc);
+          if (!is_v) {
+            named_bar_sync(1, kProdThreads);  // the previous tile's copies have all been issued
+            for (int r = pt; r < kBlockN; r += kProdThreads) {
+              const int pos = pos0 + r;
+              int src = -1;
+              if (pos < unit.kv_hi) src = __ldg(a.kv_indices + req.page0 + (pos >> shift)) * P + (pos & (P - 1));
+              sm.rowsrc[r] = src;
+            }
+            named_bar_sync(1, kProdThreads);
           }
+          if (kRows) {
+            // thread pt copies 16-byte column ch of rows r0, r0 + kRowStep, ...:
+            // the source row is read once per row and the column offset is fixed.
+            const __nv_bfloat16* base = (is_v ? a.v : a.k) + unit.kv_head * D;
+            const uint32_t dst = smem_u32(sm.kv[slot]);
+            constexpr int kRowStep = kProdThreads / kChunks;
+            const int ch = pt % kChunks;
+            const uint32_t col_off = (uint32_t)((ch >> 3) * (kTileM * 128) + ((ch & 7) << 4));
+            const size_t row_stride = (size_t)Hk * D;
+            for (int r = pt / kChunks; r < kBlockN; r += kRowStep) {
+              const int src = sm.rowsrc[r];
+              const __nv_bfloat16* g = src >= 0 ? base + (size_t)src * row_stride + ch * 8 : a.k;
+              cp_async_16(dst + r * 128 + (col_off ^ ((r & 7) << 4)), g, src >= 0 ? 16u : 0u);
+            }
+          } else {
+            // (the page-gather instance never runs this; it is kept so that its
+            // register allocation matches the measured fast build)
+            const __nv_bfloat16* base = is_v ? a.v : a.k;
+            const uint32_t dst = smem_u32(sm.kv[slot]);
+            for (int c = pt; c < kBlockN * kChunks; c += kProdThreads) {
+              const int r = c / kChunks, ch = c % kChunks;
+              const int src = sm.rowsrc[r];
+              const __nv_bfloat16* g = src >= 0 ? base + ((size_t)src * Hk + unit.kv_head) * D + ch * 8 : base;
+              cp_async_16(dst + tile_off(r, ch), g, src >= 0 ? 16u : 0u);
+            }
+          }
+          cp_async_arrive_noinc(&sm.full[slot]);
         }
-        cp_async_arrive_noinc(&sm.full[slot]);
       }
     }
     cp_async_wait<0>();
-    // Make sure no TMA write into this CTA's shared memory is still in flight at exit.
-    if (pt == 0 && n_tiles > 0) {
-      if (a.q_tma) mbar_drain(&sm.q_full, 0);
+    // Make sure no TMA write into this CTA's shared memory is still in flight at
+    // exit: only the last kSlots items and the last Q can be (every earlier one
+    // was consumed before its slot was refilled).
+    if (pt == 0) {
+      if (a.q_tma && uq > 0) mbar_drain(&sm.q_full, (uq - 1) & 1);
       if (!kRows && a.kv_tma)
-        for (int k = 2 * n_tiles - 1; k >= 0 && k >= 2 * n_tiles - kSlots; --k)
-          mbar_drain(&sm.full[k & (kSlots - 1)], (k >> 2) & 1);
+        for (int k = kc - 1; k >= 0 && k >= kc - kSlots; --k) mbar_drain(&sm.full[k & (kSlots - 1)], (k >> 2) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
@@ -274,74 +303,87 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // operands stay in uniform registers; one elected lane issues each
     // tcgen05.mma / commit. (Run from a single divergent lane, the same loop
     // cost about twice the instructions per MMA and left the tensor core idle.)
-    if (n_tiles > 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(kTileM, kBlockN, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kTileM, D, true);
-      auto wait_item = [&](int k) {
-        mbar_wait(&sm.full[k & (kSlots - 1)], (k >> 2) & 1, wc);
-        fence_proxy_async_smem();  // cp.async rows were written through the generic proxy
-        tc_fence_after();
-      };
-      // Descriptors are built once; a K-step or another buffer only moves the
-      // start address, the low 14-bit field (addr >> 4), so offsets are added in place.
-      const uint64_t dq0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
-      const uint64_t dk0 = sdesc_sw128(smem_u32(sm.kv[0]), 16, 1024);
-      const uint64_t dv0 = sdesc_sw128(smem_u32(sm.kv[0]), kBlockN * 128, 1024);
-      constexpr uint32_t kQStep = (kTileM * D * 2) >> 4;      // one Q tile
-      constexpr uint32_t kSlotStep = (kBlockN * D * 2) >> 4;  // one K/V slot
-      auto issue_s = [&](int i, int j) {
-        const uint64_t bq = dq0 + i * kQStep, bk = dk0 + ((2 * j) & (kSlots - 1)) * kSlotStep;
+    constexpr uint32_t idesc_s = idesc_bf16_f32(kTileM, kBlockN, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(kTileM, D, true);
+    auto wait_item = [&](int k) {
+      mbar_wait(&sm.full[k & (kSlots - 1)], (k >> 2) & 1, wc);
+      fence_proxy_async_smem();  // cp.async rows were written through the generic proxy
+      tc_fence_after();
+    };
+    // Descriptors are built once; a K-step or another buffer only moves the
+    // start address, the low 14-bit field (addr >> 4), so offsets are added in place.
+    const uint64_t dq0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
+    const uint64_t dk0 = sdesc_sw128(smem_u32(sm.kv[0]), 16, 1024);
+    const uint64_t dv0 = sdesc_sw128(smem_u32(sm.kv[0]), kBlockN * 128, 1024);
+    constexpr uint32_t kQStep = (kTileM * D * 2) >> 4;      // one Q tile
+    constexpr uint32_t kSlotStep = (kBlockN * D * 2) >> 4;  // one K/V slot
+    // S_i = Q_i K^T for the K item `item`
+    auto issue_s = [&](int i, int item) {
+      const uint64_t bq = dq0 + i * kQStep, bk = dk0 + (item & (kSlots - 1)) * kSlotStep;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
-          umma_bf16_ss_elect(tmem + i * kBlockN, bq + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
-        }
-      };
-      // O_i += P_i V_j for kv columns [64h, 64h + 64) of this tile: K-steps 4h..4h+3.
-      auto issue_pv_half = [&](int i, int j, int h) {
-        const uint64_t bv = dv0 + ((2 * j + 1) & (kSlots - 1)) * kSlotStep;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
+        umma_bf16_ss_elect(tmem + i * kBlockN, bq + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
+      }
+      umma_commit_elect(&sm.s_full[i]);
+    };
+    // O_i += P_i V for kv columns [64h, 64h + 64) of the V item `item`: K-steps 4h..4h+3.
+    // `first`: the unit's first KV tile, which overwrites O_i.
+    auto issue_pv_half = [&](int i, int item, int h, bool first) {
+      const uint64_t bv = dv0 + (item & (kSlots - 1)) * kSlotStep;
 #pragma unroll
-        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
-          umma_bf16_ts_elect(tmem + 256 + i * 128, tmem + i * kBlockN + kk * 8, bv + ((kk * 16 * 128) >> 4),
-                             idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-      };
-      mbar_wait(&sm.q_full, 0, wc);
+      for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+        umma_bf16_ts_elect(tmem + 256 + i * 128, tmem + i * kBlockN + kk * 8, bv + ((kk * 16 * 128) >> 4),
+                           idesc_o, (!first || kk > 0) ? 1u : 0u);
+    };
+    int jt = 0;  // KV tiles done by this CTA (all units): s_full / p_half phases
+    int uq = 0;  // units with keys: q_full / q_empty / o_final phases
+    for (int ui = u_begin; ui < u_end; ++ui) {
+      const int n_tiles = tiles_of(a.dv.units[ui]);
+      if (n_tiles == 0) continue;
+      mbar_wait(&sm.q_full, uq & 1, wc);
       fence_proxy_async_smem();
-      wait_item(0);
-      issue_s(0, 0);
-      umma_commit_elect(&sm.s_full[0]);
-      issue_s(1, 0);
-      umma_commit_elect(&sm.s_full[1]);
-      umma_commit_elect(&sm.empty[0]);
+      wait_item(2 * jt);
+      issue_s(0, 2 * jt);
+      issue_s(1, 2 * jt);
+      umma_commit_elect(&sm.empty[(2 * jt) & (kSlots - 1)]);
+      if (n_tiles == 1) umma_commit_elect(&sm.q_empty);
       for (int j = 0; j < n_tiles; ++j) {
+        const int jj = jt + j;  // this CTA's KV tile count: item 2jj is K, 2jj+1 is V
         const bool more = j + 1 < n_tiles;
-        mbar_wait(&sm.p_half[0][0], j & 1, wc);
-        wait_item(2 * j + 1);
-        issue_pv_half(0, j, 0);
-        mbar_wait(&sm.p_half[0][1], j & 1, wc);
+        mbar_wait(&sm.p_half[0][0], jj & 1, wc);
+        wait_item(2 * jj + 1);
+        issue_pv_half(0, 2 * jj + 1, 0, j == 0);
+        mbar_wait(&sm.p_half[0][1], jj & 1, wc);
         tc_fence_after();
-        issue_pv_half(0, j, 1);
+        issue_pv_half(0, 2 * jj + 1, 1, j == 0);
         if (more) {
-          wait_item(2 * j + 2);
-          issue_s(0, j + 1);
-          umma_commit_elect(&sm.s_full[0]);
+          wait_item(2 * jj + 2);
+          issue_s(0, 2 * jj + 2);
+        } else {
+          umma_commit_elect(&sm.o_final[0]);
         }
-        mbar_wait(&sm.p_half[1][0], j & 1, wc);
+        mbar_wait(&sm.p_half[1][0], jj & 1, wc);
         tc_fence_after();
-        issue_pv_half(1, j, 0);
-        mbar_wait(&sm.p_half[1][1], j & 1, wc);
+        issue_pv_half(1, 2 * jj + 1, 0, j == 0);
+        mbar_wait(&sm.p_half[1][1], jj & 1, wc);
         tc_fence_after();
-        issue_pv_half(1, j, 1);
-        umma_commit_elect(&sm.empty[(2 * j + 1) & (kSlots - 1)]);
+        issue_pv_half(1, 2 * jj + 1, 1, j == 0);
+        umma_commit_elect(&sm.empty[(2 * jj + 1) & (kSlots - 1)]);
         if (more) {
-          issue_s(1, j + 1);
-          umma_commit_elect(&sm.s_full[1]);
-          umma_commit_elect(&sm.empty[(2 * j + 2) & (kSlots - 1)]);
+          issue_s(1, 2 * jj + 2);
+          umma_commit_elect(&sm.empty[(2 * jj + 2) & (kSlots - 1)]);
+          if (j + 2 == n_tiles) umma_commit_elect(&sm.q_empty);
+        } else {
+          umma_commit_elect(&sm.o_final[1]);
         }
       }
-      umma_commit_elect(&sm.o_final);
-      mbar_drain(&sm.o_final, 0);  // no MMA may still run when TMEM is released
+      jt += n_tiles;
+      ++uq;
     }
+    // no MMA may still run when TMEM is released
+    umma_commit_elect(&sm.mma_done);
+    mbar_drain(&sm.mma_done, 0);
     __syncwarp();
   }
   } else {
@@ -350,149 +392,171 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const int ti = warp >> 2;          // query tile
     const int r = tid & (kTileM - 1);  // row in tile == TMEM lane
     const int ru = ti * kTileM + r;    // row in unit
-    const bool row_ok = ru < unit.rows;
-    const int pr = unit.row0 + (row_ok ? ru : 0);
-    const int t = pr / G;
-    int limit = unit.kv_hi;
-    if (a.g.causal) limit = min(limit, t + req.kv_len - req.qo_len + 1);
     const float scale = a.g.sm_scale_log2;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t s_tm = lane_base + ti * kBlockN;
     const uint32_t o_tm = lane_base + 256 + ti * 128;
-    float m = -INFINITY, l = 0.f;
-    for (int j = 0; j < n_tiles; ++j) {
-      mbar_wait(&sm.s_full[ti], j & 1, wc);
-      tc_fence_after();
-      float sv[kBlockN];
-      tmem_ld64(s_tm, sv);
-      tmem_ld64(s_tm + 64, sv + 64);
-      tmem_ld_wait();
-      const int kv0 = unit.kv_lo + j * kBlockN;
-      const bool whole = kv0 + kBlockN <= limit;
-      if (!whole) {
-#pragma unroll
-        for (int c = 0; c < kBlockN; ++c)
-          if (kv0 + c >= limit) sv[c] = -INFINITY;
+    int jt = 0, uq = 0;
+    for (int ui = u_begin; ui < u_end; ++ui) {
+      // Only what the KV loop needs stays live across it; the epilogue reads
+      // the unit again (the softmax warps run close to their register budget).
+      int n_tiles, kv_lo, limit;
+      {
+        const WorkUnit unit = a.dv.units[ui];
+        const ReqInfo req = a.dv.reqs[unit.req];
+        n_tiles = tiles_of(unit);
+        kv_lo = unit.kv_lo;
+        const int t = (unit.row0 + (ru < unit.rows ? ru : 0)) / G;
+        limit = unit.kv_hi;
+        if (a.g.causal) limit = min(limit, t + req.kv_len - req.qo_len + 1);
       }
-      // row max: four independent 3-input max chains
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < n_tiles; ++j) {
+        mbar_wait(&sm.s_full[ti], (jt + j) & 1, wc);
+        tc_fence_after();
+        float sv[kBlockN];
+        tmem_ld64(s_tm, sv);
+        tmem_ld64(s_tm + 64, sv + 64);
+        tmem_ld_wait();
+        const int kv0 = kv_lo + j * kBlockN;
+        const bool whole = kv0 + kBlockN <= limit;
+        if (!whole) {
 #pragma unroll
-      for (int c = 0; c < kBlockN; c += 8) {
-        mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c], sv[c + 1]);
-        mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c + 2], sv[c + 3]);
-        mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c + 4], sv[c + 5]);
-        mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c + 6], sv[c + 7]);
+          for (int c = 0; c < kBlockN; ++c)
+            if (kv0 + c >= limit) sv[c] = -INFINITY;
+        }
+        // row max: four independent 3-input max chains
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < kBlockN; c += 8) {
+          mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c], sv[c + 1]);
+          mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c + 2], sv[c + 3]);
+          mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c + 4], sv[c + 5]);
+          mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], sv[c + 6], sv[c + 7]);
+        }
+        const float mx = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
+        const float m_cand = mx == -INFINITY ? -INFINITY : mx * scale;
+        const bool need = m_cand > m + kRescaleThreshold;
+        const float alpha = need ? ex2(m - m_cand) : 1.f;
+        const bool rescale_o = j > 0 && __any_sync(0xffffffffu, need);
+        if (need) {
+          l *= alpha;
+          m = m_cand;
+        }
+        const float mu = m == -INFINITY ? 0.f : m;
+        // p = 2^(s * scale - m) (masked columns hold -inf and give 0), packed to
+        // bf16 and stored over S in 32-column chunks; each half of P is published
+        // as soon as it is in TMEM so the P.V MMAs can start on it.
+        const float2 scale2 = make_float2(scale, scale);
+        const float2 nmu2 = make_float2(-mu, -mu);
+        float2 rs2a = make_float2(0.f, 0.f), rs2b = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pw[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c = h * 64 + 2 * e;
+            const float2 x = ffma2(make_float2(sv[c], sv[c + 1]), scale2, nmu2);
+            float2 pp;
+            if (kPolyPer8 > 0 && ((2 * e) & 7) < kPolyPer8) {
+              pp = exp2_poly2(x);
+              if (!whole) {
+                if (sv[c] == -INFINITY) pp.x = 0.f;
+                if (sv[c + 1] == -INFINITY) pp.y = 0.f;
+              }
+            } else {
+              pp.x = ex2(x.x);
+              pp.y = ex2(x.y);
+            }
+            if (e & 1) rs2b = fadd2(rs2b, pp);
+            else rs2a = fadd2(rs2a, pp);
+            pw[e] = pack_bf16x2(pp.x, pp.y);
+          }
+          tmem_st32(s_tm + h * 32, reinterpret_cast<const float*>(pw));
+          // O_i *= alpha before the first P.V MMA of this tile adds to it (the
+          // S commit covered the previous tile's P.V). Done here, with half of
+          // S already consumed, so the rescale's registers fit beside the rest.
+          if (h == 0 && rescale_o) {
+            float ov[32];
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              tmem_ld32(o_tm + c, ov);
+              tmem_ld_wait();
+#pragma unroll
+              for (int x = 0; x < 32; ++x) ov[x] *= alpha;
+              tmem_st32(o_tm + c, ov);
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&sm.p_half[ti][h]);
+        }
+        l += (rs2a.x + rs2a.y) + (rs2b.x + rs2b.y);
       }
-      const float mx = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
-      const float m_cand = mx == -INFINITY ? -INFINITY : mx * scale;
-      const bool need = m_cand > m + kRescaleThreshold;
-      const float alpha = need ? ex2(m - m_cand) : 1.f;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        float ov[32];
+      // ---------------------------------------------------------- epilogue
+      // (the loads of O_i complete before this thread's next P arrive, so the
+      // next unit's first P.V MMA cannot overwrite O_i under them)
+      if (n_tiles > 0) {
+        mbar_wait(&sm.o_final[ti], uq & 1, wc);
+        tc_fence_after();
+      }
+      const WorkUnit unit = a.dv.units[ui];
+      const ReqInfo req = a.dv.reqs[unit.req];
+      const bool row_ok = ru < unit.rows;
+      const int pr = unit.row0 + (row_ok ? ru : 0);
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float lse2 = l > 0.f ? m + __log2f(l) : -INFINITY;
+      const int tok = req.q_start + pr / G;
+      const int h = unit.kv_head * G + pr % G;
+      if (unit.partial >= 0) {
+        float* dst = a.dv.part_o + ((size_t)unit.partial * kPrefillUnitRows + ru) * D;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
-          tmem_ld32(o_tm + c, ov);
-          tmem_ld_wait();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) ov[x] *= alpha;
-          tmem_st32(o_tm + c, ov);
-        }
-        tmem_st_wait();
-      }
-      if (need) {
-        l *= alpha;
-        m = m_cand;
-      }
-      const float mu = m == -INFINITY ? 0.f : m;
-      // p = 2^(s * scale - m) (masked columns hold -inf and give 0), packed to
-      // bf16 and stored over S in 32-column chunks; each half of P is published
-      // as soon as it is in TMEM so the P.V MMAs can start on it.
-      const float2 scale2 = make_float2(scale, scale);
-      const float2 nmu2 = make_float2(-mu, -mu);
-      float2 rs2a = make_float2(0.f, 0.f), rs2b = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pw[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = h * 64 + 2 * e;
-          const float2 x = ffma2(make_float2(sv[c], sv[c + 1]), scale2, nmu2);
-          float2 pp;
-          if (kPolyPer8 > 0 && ((2 * e) & 7) < kPolyPer8) {
-            pp = exp2_poly2(x);
-            if (!whole) {
-              if (sv[c] == -INFINITY) pp.x = 0.f;
-              if (sv[c + 1] == -INFINITY) pp.y = 0.f;
-            }
+          float ov[32];
+          if (n_tiles > 0) {
+            tmem_ld32(o_tm + c, ov);
+            tmem_ld_wait();
           } else {
-            pp.x = ex2(x.x);
-            pp.y = ex2(x.y);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) ov[x] = 0.f;
           }
-          if (e & 1) rs2b = fadd2(rs2b, pp);
-          else rs2a = fadd2(rs2a, pp);
-          pw[e] = pack_bf16x2(pp.x, pp.y);
-        }
-        tmem_st32(s_tm + h * 32, reinterpret_cast<const float*>(pw));
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&sm.p_half[ti][h]);
-      }
-      l += (rs2a.x + rs2a.y) + (rs2b.x + rs2b.y);
-    }
-    // ------------------------------------------------------------ epilogue
-    if (n_tiles > 0) {
-      mbar_wait(&sm.o_final, 0, wc);
-      tc_fence_after();
-    }
-    const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    const float lse2 = l > 0.f ? m + __log2f(l) : -INFINITY;
-    const int tok = req.q_start + t;
-    const int h = unit.kv_head * G + pr % G;
-    if (unit.partial >= 0) {
-      float* dst = a.dv.part_o + ((size_t)unit.partial * kPrefillUnitRows + ru) * D;
+          if (row_ok) {
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        float ov[32];
-        if (n_tiles > 0) {
-          tmem_ld32(o_tm + c, ov);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) ov[x] = 0.f;
-        }
-        if (row_ok) {
-#pragma unroll
-          for (int x = 0; x < 32; x += 4)
-            *reinterpret_cast<float4*>(dst + c + x) =
-                make_float4(ov[x] * inv_l, ov[x + 1] * inv_l, ov[x + 2] * inv_l, ov[x + 3] * inv_l);
-        }
-      }
-      if (row_ok) a.dv.part_lse[(size_t)unit.partial * kPrefillUnitRows + ru] = lse2;
-    } else {
-      __nv_bfloat16* dst = a.o + ((size_t)tok * a.g.num_qo_heads + h) * D;
-#pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        float ov[32];
-        if (n_tiles > 0) {
-          tmem_ld32(o_tm + c, ov);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) ov[x] = 0.f;
-        }
-        if (row_ok) {
-#pragma unroll
-          for (int x = 0; x < 32; x += 8) {
-            uint4 w;
-            w.x = pack_bf16x2(ov[x + 0] * inv_l, ov[x + 1] * inv_l);
-            w.y = pack_bf16x2(ov[x + 2] * inv_l, ov[x + 3] * inv_l);
-            w.z = pack_bf16x2(ov[x + 4] * inv_l, ov[x + 5] * inv_l);
-            w.w = pack_bf16x2(ov[x + 6] * inv_l, ov[x + 7] * inv_l);
-            *reinterpret_cast<uint4*>(dst + c + x) = w;
+            for (int x = 0; x < 32; x += 4)
+              *reinterpret_cast<float4*>(dst + c + x) =
+                  make_float4(ov[x] * inv_l, ov[x + 1] * inv_l, ov[x + 2] * inv_l, ov[x + 3] * inv_l);
           }
         }
+        if (row_ok) a.dv.part_lse[(size_t)unit.partial * kPrefillUnitRows + ru] = lse2;
+      } else {
+        __nv_bfloat16* dst = a.o + ((size_t)tok * a.g.num_qo_heads + h) * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          float ov[32];
+          if (n_tiles > 0) {
+            tmem_ld32(o_tm + c, ov);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) ov[x] = 0.f;
+          }
+          if (row_ok) {
+#pragma unroll
+            for (int x = 0; x < 32; x += 8) {
+              uint4 w;
+              w.x = pack_bf16x2(ov[x + 0] * inv_l, ov[x + 1] * inv_l);
+              w.y = pack_bf16x2(ov[x + 2] * inv_l, ov[x + 3] * inv_l);
+              w.z = pack_bf16x2(ov[x + 4] * inv_l, ov[x + 5] * inv_l);
+              w.w = pack_bf16x2(ov[x + 6] * inv_l, ov[x + 7] * inv_l);
+              *reinterpret_cast<uint4*>(dst + c + x) = w;
+            }
+          }
+        }
+        if (row_ok && a.lse) a.lse[(size_t)tok * a.g.num_qo_heads + h] = lse2;
       }
-      if (row_ok && a.lse) a.lse[(size_t)tok * a.g.num_qo_heads + h] = lse2;
+      tc_fence_before();
+      jt += n_tiles;
+      if (n_tiles > 0) ++uq;
     }
   }
   tc_fence_before();
@@ -540,7 +604,7 @@ cudaError_t launch_as(const Args& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  prefill_kernel<D, kRows><<<a.g.num_units, kThreads, smem, stream>>>(a);
+  prefill_kernel<D, kRows><<<a.g.num_ctas, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -554,7 +618,7 @@ cudaError_t launch(const Args& a, cudaStream_t stream) {
 cudaError_t launch_prefill(const LaunchGeom& g, const DeviceView& dv, const int32_t* kv_indices, const void* q,
                            const void* k, const void* v, int32_t num_pages, void* o, float* lse,
                            cudaStream_t stream) {
-  if (g.num_units == 0) return cudaSuccess;
+  if (g.num_units == 0 || g.num_ctas == 0) return cudaSuccess;
   Args a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k = static_cast<const __nv_bfloat16*>(k);

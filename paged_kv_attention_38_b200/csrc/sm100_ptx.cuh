@@ -77,10 +77,13 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 
 // Wait for the phase with parity `parity` of `bar` to complete. Returns false
 // (after recording the error) if the CTA is aborting or the time limit passed.
+// Once a CTA aborts, every later wait returns at once, so loops that keep
+// going after a failed wait end quickly.
 // The hardware suspends the thread inside each try_wait (up to 20 us) until the
 // phase completes; the abort flags and the clock are only read every 64 tries.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& ctx) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (*ctx.abort_smem) return false;  // the CTA is already giving up: do not sleep
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
@@ -129,6 +132,13 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, uint
       " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
       : "memory");
+}
+
+// Pull a tile of a tensor-map tensor into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tmap, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {

@@ -151,10 +151,31 @@ def test_planner_kinds():
 
 
 def test_longest_units_first():
-    pl = _plan(W.gqa_prefill())
+    """Decode CTAs run one unit each, handed out in index order: longest first."""
+    pl = _plan(W.paged_decode())
+    assert pl.cta_units().size == 0 and pl.num_ctas == pl.num_units
     u = pl.work_units()
     lens = u[:, 5] - u[:, 4]
     assert np.all(np.diff(lens) <= 0)
+
+
+@pytest.mark.parametrize("maker", [W.gqa_prefill, lambda: W.sparse_vs_dense(16, 2048, True), W.tiny_prefill])
+def test_persistent_prefill_schedule(maker):
+    """Prefill: min(SMs, units) persistent CTAs; every unit in exactly one CTA's
+    list, each list longest first, and the greedy balance bound: the loads
+    (KV tiles + 1 per unit) differ by at most one unit's cost."""
+    p = maker()
+    pl = _plan(p)
+    u = pl.work_units()
+    ptr = pl.cta_units()
+    assert pl.num_ctas == min(148, len(u)) == len(ptr) - 1
+    assert ptr[0] == 0 and ptr[-1] == len(u) and np.all(np.diff(ptr) >= 1)
+    cost = (u[:, 5] - u[:, 4] + 127) // 128 + 1
+    loads = np.array([cost[a:b].sum() for a, b in zip(ptr[:-1], ptr[1:])])
+    for a, b in zip(ptr[:-1], ptr[1:]):
+        assert np.all(np.diff(u[a:b, 5] - u[a:b, 4]) <= 0)
+    assert loads.max() - loads.min() <= cost.max()
+    assert loads.sum() == cost.sum()
 
 
 @pytest.mark.parametrize("mutate,status", [
