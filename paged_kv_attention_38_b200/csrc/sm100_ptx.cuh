@@ -61,32 +61,20 @@ struct WaitCtx {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no legitimate wait is near this
 
-// try_wait that lets the hardware suspend the thread (up to `hint_ns`) until
-// the phase completes, instead of spinning through the issue slots.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
 // Wait for the phase with parity `parity` of `bar` to complete. Returns false
 // (after recording the error) if the CTA is aborting or the time limit passed.
 // Once a CTA aborts, every later wait returns at once, so loops that keep
 // going after a failed wait end quickly.
-// The hardware suspends the thread inside each try_wait (up to 20 us) until the
-// phase completes; the abort flags and the clock are only read every 64 tries.
+// Each try_wait may suspend the thread for a short, hardware-chosen time and
+// returns as soon as the phase completes; the abort flags and the clock are
+// only read every 64 tries. (A try_wait given a long suspend-time hint woke
+// later after the phase completed: about 2 % slower prefill.)
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& ctx) {
   if (mbar_try_wait(bar, parity)) return true;
   if (*ctx.abort_smem) return false;  // the CTA is already giving up: do not sleep
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 63) {
       if (t0 == 0) t0 = globaltimer_ns();
       if (*ctx.abort_smem) return false;
