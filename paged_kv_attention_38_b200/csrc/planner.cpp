@@ -21,6 +21,10 @@ namespace pkv {
 
 namespace {
 
+// K/V bytes above which prefill units are ordered in L2-sized bands (L2 is
+// 126 MB on B200; Q, O and other CTAs' data share it).
+constexpr int64_t kL2BandBytes = 48ll << 20;
+
 bool is_pow2(int32_t x) { return x > 0 && (x & (x - 1)) == 0; }
 
 int ilog2(int32_t x) {
@@ -158,11 +162,40 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   s.num_slots = slots;
 
   // Longest units first: with a non-persistent grid the hardware hands out
-  // CTAs roughly in index order, so this is a greedy longest-processing-time
+  // CTAs roughly in index order, and the persistent prefill schedule below
+  // assigns units in list order, so this is a greedy longest-processing-time
   // schedule that keeps the tail short.
-  std::stable_sort(s.units.begin(), s.units.end(), [](const WorkUnit& a, const WorkUnit& b) {
+  auto longest_first = [](const WorkUnit& a, const WorkUnit& b) {
     return (a.kv_hi - a.kv_lo) > (b.kv_hi - b.kv_lo);
-  });
+  };
+  int64_t kv_bytes = 0;  // K and V bytes of the whole batch
+  for (const ReqInfo& r : s.reqs) kv_bytes += (int64_t)r.kv_len * in.num_kv_heads * (in.head_dim + in.head_dim_v) * 2;
+  if (s.kind == kKindPrefill && kv_bytes > kL2BandBytes) {
+    // When the batch's K/V does not fit in L2 beside everything else, a global
+    // longest-first order runs one unit of every (request, kv head) at a time
+    // and each unit re-reads its keys from HBM. Instead cut the work list (in
+    // (request, kv head) order) into bands of whole groups holding at least
+    // one unit per SM, longest first within a band: the units that run at the
+    // same time then share a few groups' K/V, which stays in L2.
+    std::vector<WorkUnit> out;
+    out.reserve(s.units.size());
+    size_t begin = 0;
+    while (begin < s.units.size()) {
+      size_t end = begin;
+      while (end < s.units.size()) {
+        const WorkUnit& u = s.units[end];
+        ++end;
+        const bool group_ends = end == s.units.size() || s.units[end].req != u.req || s.units[end].kv_head != u.kv_head;
+        if (group_ends && end - begin >= (size_t)num_sms) break;
+      }
+      std::stable_sort(s.units.begin() + begin, s.units.begin() + end, longest_first);
+      out.insert(out.end(), s.units.begin() + begin, s.units.begin() + end);
+      begin = end;
+    }
+    s.units.swap(out);
+  } else {
+    std::stable_sort(s.units.begin(), s.units.end(), longest_first);
+  }
 
   // Prefill runs persistent CTAs (one per SM), each over a fixed list of
   // units. Greedy list scheduling in the longest-first order above: each unit

@@ -159,11 +159,15 @@ def test_longest_units_first():
     assert np.all(np.diff(lens) <= 0)
 
 
-@pytest.mark.parametrize("maker", [W.gqa_prefill, lambda: W.sparse_vs_dense(16, 2048, True), W.tiny_prefill])
-def test_persistent_prefill_schedule(maker):
+@pytest.mark.parametrize("maker,banded", [(W.gqa_prefill, False), (lambda: W.sparse_vs_dense(16, 2048, True), True),
+                                          (W.tiny_prefill, False)])
+def test_persistent_prefill_schedule(maker, banded):
     """Prefill: min(SMs, units) persistent CTAs; every unit in exactly one CTA's
-    list, each list longest first, and the greedy balance bound: the loads
-    (KV tiles + 1 per unit) differ by at most one unit's cost."""
+    list and the greedy balance bound: the loads (KV tiles + 1 per unit)
+    differ by at most one unit's cost. Each CTA's list is longest first; when
+    the batch's K/V exceeds the L2 band size (16 x 2048 tokens x 8 kv heads:
+    134 MB) it is instead ordered band by band, i.e. by (request, kv head)
+    group, so that concurrently running units share groups."""
     p = maker()
     pl = _plan(p)
     u = pl.work_units()
@@ -172,10 +176,25 @@ def test_persistent_prefill_schedule(maker):
     assert ptr[0] == 0 and ptr[-1] == len(u) and np.all(np.diff(ptr) >= 1)
     cost = (u[:, 5] - u[:, 4] + 127) // 128 + 1
     loads = np.array([cost[a:b].sum() for a, b in zip(ptr[:-1], ptr[1:])])
+    group = u[:, 0].astype(np.int64) * p.num_kv_heads + u[:, 1]
+    # bands: whole groups in (request, kv head) order, cut once a band holds >= 148 units
+    per_group = np.bincount(group, minlength=int(group.max()) + 1)
+    band_of, band, run = np.zeros(len(per_group), np.int64), 0, 0
+    for g_, n in enumerate(per_group):
+        band_of[g_] = band
+        run += n
+        if run >= 148:
+            band, run = band + 1, 0
+    band_u = band_of[group]
     for a, b in zip(ptr[:-1], ptr[1:]):
-        assert np.all(np.diff(u[a:b, 5] - u[a:b, 4]) <= 0)
+        if banded:
+            assert np.all(np.diff(band_u[a:b]) >= 0)
+        else:
+            assert np.all(np.diff(u[a:b, 5] - u[a:b, 4]) <= 0)
     assert loads.max() - loads.min() <= cost.max()
     assert loads.sum() == cost.sum()
+    # coverage: every (req, head, row block, kv range) exactly once
+    assert len({tuple(r) for r in u[:, :6].tolist()}) == len(u)
 
 
 @pytest.mark.parametrize("mutate,status", [
