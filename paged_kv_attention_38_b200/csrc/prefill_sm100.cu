@@ -76,6 +76,7 @@ template <int D>
 struct __align__(1024) Smem {
   __nv_bfloat16 q[kTiles][kTileM * D];
   __nv_bfloat16 kv[kSlots][kBlockN * D];
+  alignas(128) uint8_t ostage[kPrefillUnitRows][128];  // epilogue staging (row gather instance): 128 B per row
   uint64_t q_full;
   uint64_t q_empty;  // the unit's last QK^T MMAs are done: Q may be overwritten
   uint64_t full[kSlots];
@@ -88,6 +89,8 @@ struct __align__(1024) Smem {
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(offsetof(Smem<64>, ostage) % 128 == 0 && offsetof(Smem<128>, ostage) % 128 == 0,
+              "16-byte shared stores into the staging rows");
 
 struct Args {
   CUtensorMap tm_q;
@@ -508,51 +511,116 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
       const float lse2 = l > 0.f ? m + __log2f(l) : -INFINITY;
       const int tok = req.q_start + pr / G;
       const int h = unit.kv_head * G + pr % G;
-      if (unit.partial >= 0) {
-        float* dst = a.dv.part_o + ((size_t)unit.partial * kPrefillUnitRows + ru) * D;
+      if constexpr (kRows) {
+        // Rows leave through this warp's staging tile in shared memory, 128 bytes
+        // of each of its 32 rows per pass, so that every global store
+        // instruction writes four whole 128-byte lines (eight lanes per row)
+        // instead of a 16-byte piece of 32 different lines. fp32 partial state
+        // (split units) takes 32 columns per pass, bf16 O 64.
+        const bool part = unit.partial >= 0;
+        char* my_dst = nullptr;
+        if (row_ok)
+          my_dst = part ? reinterpret_cast<char*>(a.dv.part_o + ((size_t)unit.partial * kPrefillUnitRows + ru) * D)
+                        : reinterpret_cast<char*>(a.o + ((size_t)tok * a.g.num_qo_heads + h) * D);
+        // this warp's 32 rows are ru & ~31 ... (ru & ~31) + 31; this thread's is lane ru & 31
+        const int rl = ru & 31;
+        const uint32_t stage = smem_u32(sm.ostage[ru & ~31]);
+        const int n_pass = part ? D / 32 : D / 64;
+        const uint32_t my_row = stage + rl * 128;
+        for (int ps = 0; ps < n_pass; ++ps) {
+          // this row's 128 bytes of the pass -> 8 swizzled 16-byte chunks
+          if (part) {
+            float ov[32];
+            if (n_tiles > 0) {
+              tmem_ld32(o_tm + ps * 32, ov);
+              tmem_ld_wait();
+            }
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          float ov[32];
-          if (n_tiles > 0) {
-            tmem_ld32(o_tm + c, ov);
-            tmem_ld_wait();
+            for (int k = 0; k < 8; ++k) {
+              uint32_t w[4];
+#pragma unroll
+              for (int x = 0; x < 4; ++x) w[x] = __float_as_uint(n_tiles > 0 ? ov[4 * k + x] * inv_l : 0.f);
+              st_shared_v4(my_row + ((k ^ (rl & 7)) << 4), w[0], w[1], w[2], w[3]);
+            }
           } else {
 #pragma unroll
-            for (int x = 0; x < 32; ++x) ov[x] = 0.f;
-          }
-          if (row_ok) {
+            for (int q = 0; q < 2; ++q) {
+              float ov[32];
+              if (n_tiles > 0) {
+                tmem_ld32(o_tm + ps * 64 + q * 32, ov);
+                tmem_ld_wait();
+              }
 #pragma unroll
-            for (int x = 0; x < 32; x += 4)
-              *reinterpret_cast<float4*>(dst + c + x) =
-                  make_float4(ov[x] * inv_l, ov[x + 1] * inv_l, ov[x + 2] * inv_l, ov[x + 3] * inv_l);
-          }
-        }
-        if (row_ok) a.dv.part_lse[(size_t)unit.partial * kPrefillUnitRows + ru] = lse2;
-      } else {
-        __nv_bfloat16* dst = a.o + ((size_t)tok * a.g.num_qo_heads + h) * D;
+              for (int k = 0; k < 4; ++k) {
+                uint32_t w[4];
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          float ov[32];
-          if (n_tiles > 0) {
-            tmem_ld32(o_tm + c, ov);
-            tmem_ld_wait();
-          } else {
-#pragma unroll
-            for (int x = 0; x < 32; ++x) ov[x] = 0.f;
-          }
-          if (row_ok) {
-#pragma unroll
-            for (int x = 0; x < 32; x += 8) {
-              uint4 w;
-              w.x = pack_bf16x2(ov[x + 0] * inv_l, ov[x + 1] * inv_l);
-              w.y = pack_bf16x2(ov[x + 2] * inv_l, ov[x + 3] * inv_l);
-              w.z = pack_bf16x2(ov[x + 4] * inv_l, ov[x + 5] * inv_l);
-              w.w = pack_bf16x2(ov[x + 6] * inv_l, ov[x + 7] * inv_l);
-              *reinterpret_cast<uint4*>(dst + c + x) = w;
+                for (int x = 0; x < 4; ++x)
+                  w[x] = n_tiles > 0 ? pack_bf16x2(ov[8 * k + 2 * x] * inv_l, ov[8 * k + 2 * x + 1] * inv_l) : 0u;
+                st_shared_v4(my_row + (((4 * q + k) ^ (rl & 7)) << 4), w[0], w[1], w[2], w[3]);
+              }
             }
           }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = 4 * it + (rl >> 3), k = rl & 7;
+            char* d = reinterpret_cast<char*>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(my_dst), rr));
+            const uint4 v = ld_shared_v4(stage + rr * 128 + ((k ^ (rr & 7)) << 4));
+            if (d) *reinterpret_cast<uint4*>(d + ps * 128 + k * 16) = v;
+          }
+          __syncwarp();
         }
-        if (row_ok && a.lse) a.lse[(size_t)tok * a.g.num_qo_heads + h] = lse2;
+        if (row_ok) {
+          if (part) a.dv.part_lse[(size_t)unit.partial * kPrefillUnitRows + ru] = lse2;
+          else if (a.lse) a.lse[(size_t)tok * a.g.num_qo_heads + h] = lse2;
+        }
+      } else {
+        if (unit.partial >= 0) {
+          float* dst = a.dv.part_o + ((size_t)unit.partial * kPrefillUnitRows + ru) * D;
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            float ov[32];
+            if (n_tiles > 0) {
+              tmem_ld32(o_tm + c, ov);
+              tmem_ld_wait();
+            } else {
+#pragma unroll
+              for (int x = 0; x < 32; ++x) ov[x] = 0.f;
+            }
+            if (row_ok) {
+#pragma unroll
+              for (int x = 0; x < 32; x += 4)
+                *reinterpret_cast<float4*>(dst + c + x) =
+                    make_float4(ov[x] * inv_l, ov[x + 1] * inv_l, ov[x + 2] * inv_l, ov[x + 3] * inv_l);
+            }
+          }
+          if (row_ok) a.dv.part_lse[(size_t)unit.partial * kPrefillUnitRows + ru] = lse2;
+        } else {
+          __nv_bfloat16* dst = a.o + ((size_t)tok * a.g.num_qo_heads + h) * D;
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            float ov[32];
+            if (n_tiles > 0) {
+              tmem_ld32(o_tm + c, ov);
+              tmem_ld_wait();
+            } else {
+#pragma unroll
+              for (int x = 0; x < 32; ++x) ov[x] = 0.f;
+            }
+            if (row_ok) {
+#pragma unroll
+              for (int x = 0; x < 32; x += 8) {
+                uint4 w;
+                w.x = pack_bf16x2(ov[x + 0] * inv_l, ov[x + 1] * inv_l);
+                w.y = pack_bf16x2(ov[x + 2] * inv_l, ov[x + 3] * inv_l);
+                w.z = pack_bf16x2(ov[x + 4] * inv_l, ov[x + 5] * inv_l);
+                w.w = pack_bf16x2(ov[x + 6] * inv_l, ov[x + 7] * inv_l);
+                *reinterpret_cast<uint4*>(dst + c + x) = w;
+              }
+            }
+          }
+          if (row_ok && a.lse) a.lse[(size_t)tok * a.g.num_qo_heads + h] = lse2;
+        }
       }
       tc_fence_before();
       jt += n_tiles;
