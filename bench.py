@@ -76,8 +76,12 @@ def attention_flops(p: W.PagedProblem) -> float:
 def decode_bytes(p: W.PagedProblem) -> float:
     """Algorithmic HBM bytes of a decode pass: K and V rows of every request once,
     Q and O (bf16), LSE (fp32) and the page indices."""
-    kv = 2 * 2 * p.num_kv_heads * p.head_dim * int(p.kv_lens.sum())
-    q = 2 * p.total_q * p.num_qo_heads * p.head_dim
+    if p.is_mla:  # one latent row (ckv | kpe) per key serves as both K and V
+        kv = 2 * (p.head_dim + p.head_dim_pe) * int(p.kv_lens.sum())
+        q = 2 * p.total_q * p.num_qo_heads * (p.head_dim + p.head_dim_pe)
+    else:
+        kv = 2 * 2 * p.num_kv_heads * p.head_dim * int(p.kv_lens.sum())
+        q = 2 * p.total_q * p.num_qo_heads * p.head_dim
     o = 2 * p.total_q * p.num_qo_heads * p.head_dim_v
     lse = 4 * p.total_q * p.num_qo_heads
     idx = 4 * len(p.kv_indices)
@@ -512,7 +516,8 @@ def run_only(args, device, flush):
     makers = {"prefill": W.gqa_prefill, "decode": W.paged_decode, "mla": W.mla_prefill,
               "decode_small": lambda: W.paged_decode(batch=32),
               "sparse": lambda: W.sparse_vs_dense(16, 2048, False),
-              "dense": lambda: W.sparse_vs_dense(16, 2048, True)}
+              "dense": lambda: W.sparse_vs_dense(16, 2048, True),
+              "mla_decode": W.mla_decode}
     c = Case(makers[args.only](), device)
     sampler = ClockSampler(device.index or 0)
     with sampler:
@@ -520,7 +525,7 @@ def run_only(args, device, flush):
     f = attention_flops(c.p)
     print(json.dumps({"only": args.only, "ms_median": med, "ms_mean": mean,
                       "tflops": f / (med * 1e-3) / 1e12,
-                      "gbs": decode_bytes(c.p) / (med * 1e-3) / 1e9 if args.only.startswith("decode") else None,
+                      "gbs": decode_bytes(c.p) / (med * 1e-3) / 1e9 if "decode" in args.only else None,
                       "units": c.plan.num_units, "merges": c.plan.num_merges,
                       "clocks": sampler.summary()}), flush=True)
 
@@ -581,7 +586,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--sweep", action="store_true", help="also run the vector-sparse vs dense sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "decode_small", "mla", "sparse", "dense"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "decode_small", "mla", "mla_decode", "sparse", "dense"], default=None,
                     help="time one workload alone (profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -110,7 +110,11 @@ PKV_API pkv_status pkv_plan_create(const int32_t* qo_indptr, const int32_t* kv_i
                            float sm_scale, const pkv_plan_options* opts, pkv_plan** out);
 
 /* Plan an absorbed-MLA batch: num_heads query heads share one latent KV
- * (ckv of width head_dim_ckv, rope key kpe of width head_dim_kpe). */
+ * (ckv of width head_dim_ckv, rope key kpe of width head_dim_kpe). A batch
+ * whose requests all have qo_len <= 1 and num_heads <= 16 is planned as MLA
+ * decode (FlashInfer 0.2 release, "Fused MLA decode kernel": one CTA streams a
+ * request's latent rows once for all its heads, split-KV + merge); any other
+ * batch runs the tensor-core MLA prefill kernel. */
 PKV_API pkv_status pkv_plan_create_mla(const int32_t* qo_indptr, const int32_t* kv_indptr, const int32_t* kv_indices,
                                const int32_t* kv_last_page_len, int32_t batch, int32_t num_heads,
                                int32_t head_dim_ckv, int32_t head_dim_kpe, int32_t page_size, int32_t causal,
@@ -180,7 +184,7 @@ PKV_API pkv_status pkv_decode_noalloc(const void* q, const void* k_cache, const 
 PKV_API pkv_status pkv_device_status(const pkv_plan* plan, void* stream, int32_t* code);
 
 /* Introspection (host only, no device access):
- *   key 0 kernel kind (0 prefill, 1 decode, 2 MLA), 1 work units, 2 merge tasks,
+ *   key 0 kernel kind (0 prefill, 1 decode, 2 MLA, 3 MLA decode), 1 work units, 2 merge tasks,
  *   3 partial slots, 4 rows per partial slot, 5 SMs planned for, 6 KV chunk,
  *   7 CTAs of the main launch (prefill: persistent CTAs, each running a fixed
  *   list of work units; decode / MLA: one CTA per work unit). */

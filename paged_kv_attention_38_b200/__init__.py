@@ -32,7 +32,7 @@ lib_path = os.environ.get("PKV_LIBRARY") or os.path.join(_HERE, "libpkv.so")
 PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED, PKV_ENOSPACE, PKV_ECUDA, PKV_EDEVICE = range(6)
 _STATUS = {0: "OK", 1: "EINVAL", 2: "EUNSUPPORTED", 3: "ENOSPACE", 4: "ECUDA", 5: "EDEVICE"}
 
-KIND_PREFILL, KIND_DECODE, KIND_MLA = 0, 1, 2
+KIND_PREFILL, KIND_DECODE, KIND_MLA, KIND_MLA_DECODE = 0, 1, 2, 3
 
 
 class PkvError(RuntimeError):

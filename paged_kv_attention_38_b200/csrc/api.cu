@@ -18,6 +18,8 @@ cudaError_t launch_decode(const LaunchGeom&, const DeviceView&, const int32_t*, 
                           const void*, void*, float*, cudaStream_t);
 cudaError_t launch_mla(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
                        const void*, const void*, void*, float*, cudaStream_t);
+cudaError_t launch_mla_decode(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
+                              const void*, const void*, void*, float*, cudaStream_t);
 cudaError_t launch_merge_tasks(const LaunchGeom&, const DeviceView&, void*, float*, cudaStream_t);
 cudaError_t launch_merge_state(const float*, const float*, const float*, const float*, float*, float*, int, int,
                                cudaStream_t);
@@ -193,7 +195,7 @@ pkv_status pkv_run(const pkv_plan* p, const void* q, const void* k_cache, const 
   if (!p) return fail(PKV_EINVAL, "plan is NULL");
   if (!p->uploaded) return fail(PKV_EINVAL, "plan not uploaded (call pkv_plan_upload)");
   const Schedule& s = p->sched;
-  if (s.kind == kKindMla) return fail(PKV_EINVAL, "MLA plan: use pkv_run_mla");
+  if (s.kind == kKindMla || s.kind == kKindMlaDecode) return fail(PKV_EINVAL, "MLA plan: use pkv_run_mla");
   if (s.units.empty()) return PKV_OK;
   if (!q || !k_cache || !v_cache || !o || !p->kv_indices) return fail(PKV_EINVAL, "NULL tensor pointer");
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
@@ -213,7 +215,7 @@ pkv_status pkv_run_mla(const pkv_plan* p, const void* q_nope, const void* q_pe, 
   if (!p) return fail(PKV_EINVAL, "plan is NULL");
   if (!p->uploaded) return fail(PKV_EINVAL, "plan not uploaded (call pkv_plan_upload)");
   const Schedule& s = p->sched;
-  if (s.kind != kKindMla) return fail(PKV_EINVAL, "not an MLA plan: use pkv_run");
+  if (s.kind != kKindMla && s.kind != kKindMlaDecode) return fail(PKV_EINVAL, "not an MLA plan: use pkv_run");
   if (s.units.empty()) return PKV_OK;
   if (!q_nope || !q_pe || !ckv_cache || !kpe_cache || !o || !p->kv_indices)
     return fail(PKV_EINVAL, "NULL tensor pointer");
@@ -221,7 +223,9 @@ pkv_status pkv_run_mla(const pkv_plan* p, const void* q_nope, const void* q_pe, 
     return fail(PKV_EINVAL, "tensor pointers must be 16-byte aligned");
   if (num_pages <= 0) return fail(PKV_EINVAL, "num_pages must be positive");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_mla(s.geom, p->dv, p->kv_indices, q_nope, q_pe, ckv_cache, kpe_cache, o, lse, st);
+  cudaError_t e = s.kind == kKindMlaDecode
+                      ? launch_mla_decode(s.geom, p->dv, p->kv_indices, q_nope, q_pe, ckv_cache, kpe_cache, o, lse, st)
+                      : launch_mla(s.geom, p->dv, p->kv_indices, q_nope, q_pe, ckv_cache, kpe_cache, o, lse, st);
   if (e == cudaSuccess) e = launch_merge_tasks(s.geom, p->dv, o, lse, st);
   if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
   return PKV_OK;

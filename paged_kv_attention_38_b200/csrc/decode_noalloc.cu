@@ -320,6 +320,10 @@ cudaError_t launch(const NaArgs& a, int batch, cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(noalloc_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // all of the unified L1 / shared array as shared memory, so two CTAs fit per SM
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(noalloc_decode_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured = true;
   }

@@ -79,18 +79,27 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
   const int n = (unit.kv_hi - unit.kv_lo + kTile - 1) / kTile;
   const uint32_t sbase = smem_u32(smem);
 
+  // All page-table reads of a tile are issued before its copies: a read inside
+  // the copy loop would wait for the previous copy to be issued (the copies
+  // are ordered memory operations), serialising one global read per copy.
+  constexpr int kPerThread = kTile * kChunks / kThreads;
+  static_assert(kTile * kChunks % kThreads == 0, "whole copies per thread");
   auto load_tile = [&](int j, int stage) {
     const uint32_t kdst = sbase + stage * 2 * kTileBytes;
     const uint32_t vdst = kdst + kTileBytes;
-    for (int c = tid; c < kTile * kChunks; c += kThreads) {
+    int page[kPerThread];
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) {
+      const int pos = unit.kv_lo + j * kTile + (tid + i * kThreads) / kChunks;
+      page[i] = pos < unit.kv_hi ? __ldg(a.kv_indices + req.page0 + (pos >> shift)) : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) {
+      const int c = tid + i * kThreads;
       const int r = c / kChunks, ch = c % kChunks;
       const int pos = unit.kv_lo + j * kTile + r;
-      const bool ok = pos < unit.kv_hi;
-      size_t off = 0;
-      if (ok) {
-        const int page = __ldg(a.kv_indices + req.page0 + (pos >> shift));
-        off = (((size_t)page * P + (pos & (P - 1))) * Hk + unit.kv_head) * D + ch * 8;
-      }
+      const bool ok = page[i] >= 0;
+      const size_t off = ok ? (((size_t)page[i] * P + (pos & (P - 1))) * Hk + unit.kv_head) * D + ch * 8 : 0;
       cp_async_16(kdst + kv_off<D>(r, ch), a.k + off, ok ? 16u : 0u);
       cp_async_16(vdst + kv_off<D>(r, ch), a.v + off, ok ? 16u : 0u);
     }
@@ -267,6 +276,9 @@ cudaError_t launch(const Args& a, cudaStream_t stream) {
   const size_t smem = pipe > comb ? pipe : comb;
   auto kern = decode_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // all of the unified L1 / shared array as shared memory, so two CTAs fit per SM
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   kern<<<a.g.num_units, kThreads, smem, stream>>>(a);
   return cudaGetLastError();

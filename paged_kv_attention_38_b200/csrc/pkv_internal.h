@@ -14,7 +14,7 @@ constexpr int kBlockN = 128;   // KV slots per prefill KV tile
 constexpr int kDecodeRows = 16;  // packed rows per decode unit (mma.sync M)
 constexpr int kDecodeTileN = 64;  // KV slots per decode pipeline stage
 
-enum KernelKind : int32_t { kKindPrefill = 0, kKindDecode = 1, kKindMla = 2 };
+enum KernelKind : int32_t { kKindPrefill = 0, kKindDecode = 1, kKindMla = 2, kKindMlaDecode = 3 };
 
 // One CTA's worth of attention: packed query rows [row0, row0 + rows) of
 // request `req` for kv head `kv_head`, over keys [kv_lo, kv_hi).

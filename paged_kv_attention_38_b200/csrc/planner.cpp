@@ -90,7 +90,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   }
 
   // ---- kernel choice
-  if (mla) s.kind = kKindMla;
+  if (mla) s.kind = (max_qo <= 1 && in.num_qo_heads <= kDecodeRows) ? kKindMlaDecode : kKindMla;
   else if (max_qo <= 1 && group <= kDecodeRows) s.kind = kKindDecode;
   else s.kind = kKindPrefill;
 
@@ -99,7 +99,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   // Rows per work unit: decode packs one token's group of heads into an mma.sync
   // tile; prefill units hold two 128-row tensor-core tiles that share K/V; MLA
   // packs tokens x heads the same way with one latent "kv head".
-  const int32_t rows_per_tile = s.kind == kKindDecode ? kDecodeRows
+  const int32_t rows_per_tile = (s.kind == kKindDecode || s.kind == kKindMlaDecode) ? kDecodeRows
                                 : s.kind == kKindMla  ? kMlaUnitRows
                                                       : kPrefillUnitRows;
 
@@ -124,16 +124,34 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   }
 
   // ---- split-KV chunk
-  const int32_t align = s.kind == kKindDecode ? kDecodeTileN : s.kind == kKindMla ? 64 : kBlockN;
+  const int32_t align = (s.kind == kKindDecode || s.kind == kKindMlaDecode) ? kDecodeTileN
+                        : s.kind == kKindMla                               ? 64
+                                                                           : kBlockN;
   int64_t chunk = 0;  // 0 = no split
   if (!in.disable_split_kv) {
     if (in.kv_chunk > 0) {
       chunk = round_up(in.kv_chunk, align);
-    } else if (s.kind == kKindDecode) {
+    } else if (s.kind == kKindDecode || s.kind == kKindMlaDecode) {
       // Decode is HBM-bound: aim for ~8 units per SM so the tail is short; a
       // chunk below 512 keys would spend more on partial state than it saves.
       chunk = round_up(std::max<int64_t>(512, total_cost / ((int64_t)num_sms * 8)), align);
       chunk = std::min<int64_t>(chunk, 4096);
+      // Wave quantisation: units run two CTAs per SM in waves of 2 x SMs, and
+      // a last wave that is nearly empty costs as much as a full one. Among
+      // chunks up to 2x the first guess take the one with the smallest
+      // (waves x chunk), the time model of equal, full-chunk units.
+      const int64_t wave = 2 * (int64_t)num_sms;
+      int64_t best = chunk, best_t = INT64_MAX;
+      for (int64_t c = chunk; c <= 2 * chunk; c += align) {
+        int64_t units = 0;
+        for (const Tile& t : tiles) units += (t.kv_need + c - 1) / c;
+        const int64_t t_est = (units + wave - 1) / wave * std::min<int64_t>(c, max_need);
+        if (t_est < best_t) {
+          best_t = t_est;
+          best = c;
+        }
+      }
+      chunk = best;
     } else {
       // Prefill: one CTA per SM at a time; split only when a single tile is
       // longer than the average work per SM.

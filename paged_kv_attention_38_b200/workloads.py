@@ -275,6 +275,15 @@ def paged_decode(batch: int = 128, lo: int = 1024, hi: int = 8192, shard: int = 
                         causal=False, seed=seed)
 
 
+def mla_decode(batch: int = 64, lo: int = 1024, hi: int = 8192, shard: int = 0) -> PagedProblem:
+    """Absorbed MLA decode: one query token per request, 16 heads, ckv 512 + kpe 64,
+    page_size 1 (slots scattered over the pool), kv_len ~ U[lo, hi], sm_scale 1/sqrt(192)."""
+    seed = SEED_BASE + 6 + 10000 * shard
+    kv = uniform_lengths(batch, lo, hi, _gen(seed + 7))
+    return make_mla_problem("mla_paged_decode_h16_ckv512_kpe64_ps1", [1] * batch, kv, num_heads=16,
+                            causal=False, seed=seed)
+
+
 def mla_prefill(batch: int = 4, lo: int = 256, hi: int = 2048, shard: int = 0) -> PagedProblem:
     """Absorbed MLA causal paged prefill, 16 heads, ckv 512 + kpe 64, page_size 1,
     sm_scale 1/sqrt(192) (h16/ckv512/kpe64/ps1)."""

@@ -148,6 +148,10 @@ def test_planner_kinds():
     pl = pkv.plan_mla(m.qo_indptr, m.kv_indptr, None, m.kv_last_page_len, 16, 512, 64, 1, True,
                       m.sm_scale, upload=False, num_sms=148)
     assert pl.kind == pkv.KIND_MLA
+    d = W.mla_decode()
+    pl = pkv.plan_mla(d.qo_indptr, d.kv_indptr, None, d.kv_last_page_len, 16, 512, 64, 1, False,
+                      d.sm_scale, upload=False, num_sms=148)
+    assert pl.kind == pkv.KIND_MLA_DECODE and pl.info(4) == 16  # 16 rows (heads) per partial slot
 
 
 def test_longest_units_first():

@@ -283,6 +283,36 @@ def test_mla_split_kv():
     assert_parity(o, lse, *oracle_mla(p), what="mla split")
 
 
+MLA_DECODE = [
+    # kv_lens, heads, page, forced kv chunk (0 = planner's)
+    ([1, 63, 64, 65, 700, 3000], 16, 1, 0),   # ragged, the longest request split
+    ([0, 5, 129, 1000], 8, 1, 64),            # fewer heads than MMA rows, an empty request, every request split
+    ([40, 300], 16, 16, 0),                   # page_size 16
+]
+
+
+@pytest.mark.parametrize("case", MLA_DECODE, ids=lambda c: f"h{c[1]}_p{c[2]}_k{c[3]}")
+def test_mla_decode_small(case):
+    """MLA decode (one query token per request, non-causal) through the decode kernel."""
+    kv, h, ps, chunk = case
+    p = W.make_mla_problem("mla_dec", [1] * len(kv), kv, num_heads=h, page_size=ps, causal=False,
+                           seed=zlib.crc32(str(case).encode()) % 10000)
+    o, lse, pl = gpu_run_mla(p, **({"kv_chunk": chunk} if chunk else {}))
+    assert pl.kind == pkv.KIND_MLA_DECODE
+    if chunk:
+        assert pl.num_merges > 0
+    assert_parity(o, lse, *oracle_mla(p), what=f"mla decode {case}")
+
+
+@pytest.mark.slow
+def test_mla_decode_full_size():
+    """h16/ckv512/kpe64/ps1 decode, batch 64, kv_len U[1024, 8192], in the bench's launch
+    configuration: every row (64 tokens x 16 heads) against the oracle."""
+    p = W.mla_decode()
+    o, lse, _ = gpu_run_mla(p)
+    assert_parity(o, lse, *oracle_mla(p), what="mla decode full")
+
+
 @pytest.mark.slow
 def test_mla_full_size_sampled():
     """h16/ckv512/kpe64/ps1, batch 4, lengths U[256, 2048]: sampled rows of every request."""
