@@ -152,6 +152,30 @@ PKV_API pkv_status pkv_merge_state(const float* o_a, const float* lse_a, const f
 PKV_API pkv_status pkv_merge_states(const float* o_parts, const float* lse_parts, int32_t num, int32_t rows,
                             int32_t dim, void* o_out, float* lse_out, void* stream);
 
+/* Append new K/V rows to the paged cache (FlashInfer 0.2 release, "KV-Cache
+ * append optimization": parallel over the new elements, not over requests;
+ * positions as in the documentation's get_batch_indices_positions).
+ * The page table (kv_indptr [batch+1], kv_indices, kv_last_page_len [batch];
+ * all DEVICE int32) is the table AFTER the append: request b's new rows,
+ * k_new / v_new rows append_indptr[b] .. append_indptr[b+1] - 1 (DEVICE int32
+ * [batch+1], nnz = append_indptr[batch] rows in total), are written to its last
+ * positions kv_len - n .. kv_len - 1 (n = its row count), i.e. page
+ * kv_indices[kv_indptr[b] + pos / page_size], slot pos % page_size.
+ * k_new [nnz, num_kv_heads, head_dim], v_new [nnz, num_kv_heads, head_dim_v]:
+ * DEVICE bf16 (any 2-byte type: bytes are copied unchanged). k_cache
+ * [num_pages, page_size, num_kv_heads, head_dim], v_cache likewise with
+ * head_dim_v: DEVICE, updated in place; every other slot is left untouched.
+ * MLA caches fit the same call with num_kv_heads 1: k = ckv (512), v = kpe (64).
+ * Head dims must be multiples of 8 and pointers 16-byte aligned.
+ * A row whose position falls outside its request, or whose page id is not in
+ * [0, num_pages), is skipped and, if `status` (DEVICE int32, may be NULL) is
+ * given, sets *status = 1. Launch only: no allocation, no synchronisation. */
+PKV_API pkv_status pkv_append_kv(const void* k_new, const void* v_new, const int32_t* append_indptr, int64_t nnz,
+                                 const int32_t* kv_indptr, const int32_t* kv_indices,
+                                 const int32_t* kv_last_page_len, int32_t batch, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t head_dim_v, int32_t page_size, int32_t num_pages,
+                                 void* k_cache, void* v_cache, int32_t* status, void* stream);
+
 /* Paged decode (one query token per request) for callers that cannot allocate
  * device memory: code under an allocator that forbids new device allocations
  * (a fixed pool, an embedded host that only registers buffers at start-up) or

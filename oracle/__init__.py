@@ -11,6 +11,7 @@ golden example and invariants); none is "parity unpinned".
 """
 from .paged_ref import (  # noqa: F401
     LN2,
+    append_paged_kv,
     attend,
     gather_pages,
     kv_lengths,

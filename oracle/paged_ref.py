@@ -31,6 +31,10 @@ What it computes, and where the pages say so
 * Merging attention states (documentation, "Attention States and Recursive
   Attention", "Merge Attention States"): two partial results over disjoint key
   sets combine by their log-sum-exp.
+* Appending new K/V rows to the paged cache (FlashInfer 0.2 release, "KV-Cache
+  append optimization"; documentation, ``get_batch_indices_positions``): the
+  page table given is the one after the append, so request ``b``'s ``n`` new
+  rows take its last ``n`` positions ``kv_len - n .. kv_len - 1``.
 
 Readings where the pages are silent (each pinned by a test)
 ------------------------------------------------------------
@@ -255,3 +259,30 @@ def merge_states(os, lses):
     for o_i, l_i in zip(os[1:], lses[1:]):
         o, lse = merge_state(o, lse, o_i, l_i)
     return o, lse
+
+
+def append_paged_kv(k_cache, v_cache, k_new, v_new, append_indptr, kv_indptr, kv_indices, kv_last_page_len,
+                    page_size: int):
+    """Return copies of the K and V pools with the new rows written in.
+
+    ``k_new``/``v_new`` ``[nnz, Hk, D]`` hold request ``b``'s new rows at
+    ``append_indptr[b]:append_indptr[b+1]``. With the page table after the
+    append, request ``b`` has ``kv_len`` positions and its ``n`` new rows are
+    positions ``kv_len - n + i``; position ``p`` lives in page
+    ``kv_indices[kv_indptr[b] + p // page_size]``, slot ``p % page_size``.
+    Plain loops, one row at a time; values are copied unchanged.
+    """
+    k_out = k_cache.clone() if hasattr(k_cache, "clone") else np.array(k_cache, copy=True)
+    v_out = v_cache.clone() if hasattr(v_cache, "clone") else np.array(v_cache, copy=True)
+    kv_len = kv_lengths(kv_indptr, kv_last_page_len, page_size)
+    for b in range(len(kv_last_page_len)):
+        a0, a1 = int(append_indptr[b]), int(append_indptr[b + 1])
+        n = a1 - a0
+        assert 0 <= n <= kv_len[b], "more new rows than the request's length"
+        for i in range(n):
+            pos = int(kv_len[b]) - n + i
+            page = int(kv_indices[int(kv_indptr[b]) + pos // page_size])
+            slot = pos % page_size
+            k_out[page, slot] = k_new[a0 + i]
+            v_out[page, slot] = v_new[a0 + i]
+    return k_out, v_out

@@ -68,6 +68,7 @@ _SIGS = {
     "pkv_plan_work_units": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
     "pkv_plan_merge_tasks": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
     "pkv_plan_cta_units": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
+    "pkv_append_kv": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P, _P, _P] + [ctypes.c_int32] * 6 + [_P, _P, _P, _P]),
     "pkv_plan_destroy": (None, [_P]),
     "pkv_last_error": (ctypes.c_char_p, []),
     "pkv_version": (ctypes.c_char_p, []),
@@ -294,6 +295,31 @@ def merge_state(o_a, lse_a, o_b, lse_b, stream=None):
     _check(load_library().pkv_merge_state(o_a.data_ptr(), lse_a.data_ptr(), o_b.data_ptr(), lse_b.data_ptr(),
                                           o.data_ptr(), lse.data_ptr(), rows, dim, _stream_ptr(stream)))
     return o, lse
+
+
+def append_kv(k_new, v_new, append_indptr, kv_indptr, kv_indices, kv_last_page_len, k_cache, v_cache,
+              status=None, stream=None):
+    """``pkv_append_kv``: write new rows ``k_new`` / ``v_new`` ``[nnz, Hk, D]`` into the
+    page pools ``[num_pages, page_size, Hk, D]`` in place, at the last positions of
+    each request under the page table after the append (all index arrays int32 on
+    the device). ``status``: optional int32 device tensor set to 1 on a bad row."""
+    import torch
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check_tensor(t, n)
+        if t.element_size() != 2:
+            raise ValueError(f"{n} must hold 2-byte elements")
+    for t, n in ((append_indptr, "append_indptr"), (kv_indptr, "kv_indptr"), (kv_indices, "kv_indices"),
+                 (kv_last_page_len, "kv_last_page_len")):
+        _check_tensor(t, n, torch.int32)
+    if k_cache.dim() == 3:  # MLA pools [num_pages, page_size, D]: one latent "head"
+        k_cache, v_cache = k_cache.unsqueeze(2), v_cache.unsqueeze(2)
+        k_new, v_new = k_new.reshape(k_new.shape[0], 1, -1), v_new.reshape(v_new.shape[0], 1, -1)
+    num_pages, page_size, hk, d = k_cache.shape
+    _check(load_library().pkv_append_kv(
+        k_new.data_ptr(), v_new.data_ptr(), append_indptr.data_ptr(), int(k_new.shape[0]), kv_indptr.data_ptr(),
+        kv_indices.data_ptr(), kv_last_page_len.data_ptr(), int(kv_last_page_len.shape[0]), hk, d,
+        int(v_cache.shape[-1]), page_size, num_pages, k_cache.data_ptr(), v_cache.data_ptr(),
+        status.data_ptr() if status is not None else None, _stream_ptr(stream)))
 
 
 def merge_states(o_parts, lse_parts, stream=None):

@@ -234,3 +234,18 @@ def test_upload_rejects_bad_workspace():
     assert lib.pkv_run(pl.handle, 16, 16, 16, 1, 16, 16, None) == pkv.PKV_EINVAL
     assert lib.pkv_merge_state(None, None, None, None, None, None, 4, 0, None) == pkv.PKV_EINVAL
     assert lib.pkv_merge_states(None, None, 0, 4, 8, None, None, None) == pkv.PKV_EINVAL
+
+
+def test_append_host_validation():
+    """pkv_append_kv rejects bad arguments on the host, before any launch."""
+    lib = pkv.load_library()
+    one = ctypes.c_int32(0)
+    p = ctypes.cast(ctypes.pointer(one), ctypes.c_void_p)  # a host address: never dereferenced on these paths
+    args = lambda nnz, hk, d, dv, ps, pages, ptr: (ptr, ptr, ptr, nnz, ptr, ptr, ptr, 1, hk, d, dv, ps, pages,
+                                                  ptr, ptr, None, None)
+    assert lib.pkv_append_kv(*args(0, 1, 64, 64, 16, 4, p)) == pkv.PKV_OK            # nothing to append
+    assert lib.pkv_append_kv(*args(-1, 1, 64, 64, 16, 4, p)) == pkv.PKV_EINVAL
+    assert lib.pkv_append_kv(*args(4, 1, 12, 64, 16, 4, p)) == pkv.PKV_EUNSUPPORTED  # head_dim not a multiple of 8
+    assert lib.pkv_append_kv(*args(4, 1, 64, 64, 0, 4, p)) == pkv.PKV_EINVAL         # page_size 0
+    assert lib.pkv_append_kv(*args(4, 1, 64, 64, 16, 4, None)) == pkv.PKV_EINVAL     # NULL pointers
+    assert b"NULL" in lib.pkv_last_error()

@@ -327,3 +327,63 @@ def test_mla_full_size_sampled():
                                                    p.sm_scale, b, pos)
         rows = [int(p.qo_indptr[b]) + x for x in pos]
         assert_parity(o[rows], lse[rows], o_r, l_r, what=f"mla req {b}")
+
+
+# --------------------------------------------------------------------------- paged KV append
+
+APPEND = [
+    # kv lengths after the append, new rows per request, kv heads, head dims (k, v), page size
+    ([37, 1, 130, 16, 0], [5, 1, 130, 16, 0], 2, (128, 128), 16),   # prefill-sized and decode-sized appends
+    ([9, 300], [1, 77], 8, (64, 64), 1),                             # vector-sparse pool
+    ([200, 65], [1, 1], 1, (512, 64), 1),                            # MLA latent rows: k = ckv, v = kpe
+]
+
+
+@pytest.mark.parametrize("case", APPEND, ids=lambda c: f"hk{c[2]}_d{c[3][0]}_p{c[4]}")
+def test_append_kv_bitwise(case):
+    kv_after, n_new, hk, (dk, dv), ps = case
+    g = np.random.default_rng(zlib.crc32(str(case).encode()))
+    kv_after, n_new = np.array(kv_after), np.array(n_new)
+    n_pages = (kv_after + ps - 1) // ps
+    pool = int(n_pages.sum()) + 5
+    kv_indptr = np.concatenate([[0], np.cumsum(n_pages)]).astype(np.int32)
+    kv_indices = g.permutation(pool)[: int(n_pages.sum())].astype(np.int32)
+    last = np.where(n_pages > 0, kv_after - (n_pages - 1) * ps, 0).astype(np.int32)
+    append_indptr = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+    nnz = int(n_new.sum())
+    k_cache = torch.from_numpy(g.standard_normal((pool, ps, hk, dk))).to(torch.bfloat16)
+    v_cache = torch.from_numpy(g.standard_normal((pool, ps, hk, dv))).to(torch.bfloat16)
+    k_new = torch.from_numpy(g.standard_normal((nnz, hk, dk))).to(torch.bfloat16)
+    v_new = torch.from_numpy(g.standard_normal((nnz, hk, dv))).to(torch.bfloat16)
+    k_ref, v_ref = oracle.append_paged_kv(k_cache, v_cache, k_new, v_new, append_indptr, kv_indptr, kv_indices,
+                                          last, ps)
+    kd, vd = k_cache.cuda(), v_cache.cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ii = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    pkv.append_kv(k_new.cuda(), v_new.cuda(), ii(append_indptr), ii(kv_indptr), ii(kv_indices), ii(last), kd, vd,
+                  status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(kd.cpu(), k_ref) and torch.equal(vd.cpu(), v_ref)
+
+
+def test_append_kv_reports_rows_without_slot():
+    """A request given more new rows than its table holds: those rows are
+    skipped and reported, every other row is written."""
+    ps, hk, d = 16, 1, 64
+    kv_after, n_new = np.array([20, 3]), np.array([2, 5])   # request 1 holds 3 positions, gets 5 rows
+    n_pages = (kv_after + ps - 1) // ps
+    kv_indptr = np.concatenate([[0], np.cumsum(n_pages)]).astype(np.int32)
+    kv_indices = np.arange(int(n_pages.sum()), dtype=np.int32)
+    last = (kv_after - (n_pages - 1) * ps).astype(np.int32)
+    append_indptr = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+    k_cache = torch.zeros(int(n_pages.sum()), ps, hk, d, dtype=torch.bfloat16, device="cuda")
+    v_cache = torch.zeros_like(k_cache)
+    k_new = torch.ones(7, hk, d, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ii = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    pkv.append_kv(k_new, k_new, ii(append_indptr), ii(kv_indptr), ii(kv_indices), ii(last), k_cache, v_cache,
+                  status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1
+    assert int(k_cache.float().sum().item()) == (2 + 3) * hk * d     # request 0's two rows + request 1's three

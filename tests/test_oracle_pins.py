@@ -464,3 +464,98 @@ def test_merge_pin_catches_natural_log_merge(monkeypatch):
     case = [c for c in _golden_cases() if c["kind"] == "merge"][0]
     with pytest.raises(AssertionError):
         test_golden_hand_worked(case)
+
+
+# --------------------------------------------------------------------------- paged KV append
+
+def _append_case(seed, page_size=4, hk=2, d=8):
+    """Lengths after the append, new-row counts, a permuted pool with spare pages."""
+    g = np.random.default_rng(seed)
+    kv_after = np.array([5, 1, 9, 12, 0], dtype=np.int64)
+    n_new = np.array([2, 1, 9, 3, 0], dtype=np.int64)
+    n_pages = (kv_after + page_size - 1) // page_size
+    kv_indptr = np.concatenate([[0], np.cumsum(n_pages)]).astype(np.int32)
+    pool = int(n_pages.sum()) + 3
+    kv_indices = g.permutation(pool)[: int(n_pages.sum())].astype(np.int32)
+    last = np.where(n_pages > 0, kv_after - (n_pages - 1) * page_size, 0).astype(np.int32)
+    append_indptr = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+    nnz = int(n_new.sum())
+    k_new = torch.from_numpy(g.standard_normal((nnz, hk, d))).to(torch.bfloat16)
+    v_new = torch.from_numpy(g.standard_normal((nnz, hk, d))).to(torch.bfloat16)
+    return dict(kv_after=kv_after, n_new=n_new, kv_indptr=kv_indptr, kv_indices=kv_indices, last=last,
+                append_indptr=append_indptr, k_new=k_new, v_new=v_new, pool=pool, page_size=page_size, hk=hk, d=d)
+
+
+def test_append_round_trip_through_gather():
+    """Append into an all-zero pool, then read each request back in order with
+    gather_pages (a separate, pinned path): positions kv_len - n .. kv_len - 1
+    hold the new rows in order, every other position is still zero."""
+    c = _append_case(1)
+    z = torch.zeros((c["pool"], c["page_size"], c["hk"], c["d"]), dtype=torch.bfloat16)
+    k, v = oracle.append_paged_kv(z, z, c["k_new"], c["v_new"], c["append_indptr"], c["kv_indptr"],
+                                  c["kv_indices"], c["last"], c["page_size"])
+    for b, (L, n) in enumerate(zip(c["kv_after"], c["n_new"])):
+        for cache, new in ((k, c["k_new"]), (v, c["v_new"])):
+            rows = oracle.gather_pages(cache, c["kv_indptr"], c["kv_indices"], c["last"], c["page_size"], b)
+            assert rows.shape[0] == L
+            a0 = int(c["append_indptr"][b])
+            assert np.array_equal(rows[L - n:], new[a0:a0 + n].float().numpy())
+            assert not np.any(rows[:L - n])
+
+
+def test_append_in_two_steps_equals_one():
+    """Appending the new rows in two batches (page table growing in between)
+    writes the same pool as one append of all of them."""
+    c = _append_case(2)
+    P = c["page_size"]
+    base = torch.from_numpy(np.random.default_rng(9).standard_normal(
+        (c["pool"], P, c["hk"], c["d"]))).to(torch.bfloat16)
+    k1, _ = oracle.append_paged_kv(base, base, c["k_new"], c["v_new"], c["append_indptr"], c["kv_indptr"],
+                                   c["kv_indices"], c["last"], P)
+    # first step: each request gets the first half of its rows, with the table truncated accordingly
+    first = c["n_new"] // 2
+    second = c["n_new"] - first
+    mid_len = c["kv_after"] - second
+    mid_pages = (mid_len + P - 1) // P
+    mid_indptr = np.concatenate([[0], np.cumsum(mid_pages)]).astype(np.int32)
+    mid_indices = np.concatenate([c["kv_indices"][c["kv_indptr"][b]:c["kv_indptr"][b] + mid_pages[b]]
+                                  for b in range(len(mid_len))]).astype(np.int32)
+    mid_last = np.where(mid_pages > 0, mid_len - (mid_pages - 1) * P, 0).astype(np.int32)
+    sel1 = np.concatenate([np.arange(c["append_indptr"][b], c["append_indptr"][b] + first[b])
+                           for b in range(len(first))]).astype(np.int64)
+    sel2 = np.concatenate([np.arange(c["append_indptr"][b] + first[b], c["append_indptr"][b + 1])
+                           for b in range(len(first))]).astype(np.int64)
+    ind1 = np.concatenate([[0], np.cumsum(first)]).astype(np.int32)
+    ind2 = np.concatenate([[0], np.cumsum(second)]).astype(np.int32)
+    ka, _ = oracle.append_paged_kv(base, base, c["k_new"][sel1], c["v_new"][sel1], ind1, mid_indptr, mid_indices,
+                                   mid_last, P)
+    kb, _ = oracle.append_paged_kv(ka, ka, c["k_new"][sel2], c["v_new"][sel2], ind2, c["kv_indptr"],
+                                   c["kv_indices"], c["last"], P)
+    assert torch.equal(k1, kb)
+
+
+def test_append_touches_only_new_slots():
+    """Slots outside the appended positions keep their old bytes (unused pool
+    pages included)."""
+    c = _append_case(3)
+    P = c["page_size"]
+    base = torch.full((c["pool"], P, c["hk"], c["d"]), 7.0, dtype=torch.bfloat16)
+    k, _ = oracle.append_paged_kv(base, base, c["k_new"], c["v_new"], c["append_indptr"], c["kv_indptr"],
+                                  c["kv_indices"], c["last"], P)
+    written = np.zeros((c["pool"], P), dtype=bool)
+    for b, (L, n) in enumerate(zip(c["kv_after"], c["n_new"])):
+        for pos in range(L - n, L):
+            written[c["kv_indices"][c["kv_indptr"][b] + pos // P], pos % P] = True
+    assert int(written.sum()) == int(c["n_new"].sum())
+    assert torch.all(k[torch.from_numpy(~written)] == 7.0)
+
+
+def test_append_pin_catches_off_by_one(monkeypatch):
+    """A planted off-by-one in the oracle's position rule fails the round-trip pin."""
+    real = paged_ref.kv_lengths
+    monkeypatch.setattr(paged_ref, "kv_lengths", lambda *a: real(*a) + 1)
+    with pytest.raises(AssertionError):
+        try:
+            test_append_round_trip_through_gather()
+        except IndexError as e:  # a shifted position may also run off the page list
+            raise AssertionError(str(e))
