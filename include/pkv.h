@@ -147,6 +147,15 @@ PKV_API pkv_status pkv_run_mla(const pkv_plan* plan, const void* q_nope, const v
 PKV_API pkv_status pkv_merge_state(const float* o_a, const float* lse_a, const float* o_b, const float* lse_b,
                            float* o_out, float* lse_out, int32_t rows, int32_t dim, void* stream);
 
+/* The same merge on bf16 outputs, as two attention runs produce them (FlashInfer
+ * 0.7.4 documentation, flashinfer.cascade: "Merge Attention States" and
+ * "Cascade Attention": a batch sharing a KV prefix attends to the prefix once
+ * and to each request's own pages once, and the two states are merged).
+ * o_a, o_b, o_out: DEVICE bf16 [rows, dim]; lse_*: DEVICE fp32 [rows], base 2.
+ * Arithmetic in fp32; o_out / lse_out may alias o_a / lse_a. dim <= 1024. */
+PKV_API pkv_status pkv_merge_state_bf16(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                                        void* o_out, float* lse_out, int32_t rows, int32_t dim, void* stream);
+
 /* Merge `num` states (DEVICE fp32 o_parts [num, rows, dim], lse_parts [num, rows])
  * into bf16 o_out [rows, dim] and fp32 lse_out [rows]. dim <= 1024. */
 PKV_API pkv_status pkv_merge_states(const float* o_parts, const float* lse_parts, int32_t num, int32_t rows,

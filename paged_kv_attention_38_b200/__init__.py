@@ -68,6 +68,7 @@ _SIGS = {
     "pkv_plan_work_units": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
     "pkv_plan_merge_tasks": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
     "pkv_plan_cta_units": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
+    "pkv_merge_state_bf16": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
     "pkv_append_kv": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P, _P, _P] + [ctypes.c_int32] * 6 + [_P, _P, _P, _P]),
     "pkv_plan_destroy": (None, [_P]),
     "pkv_last_error": (ctypes.c_char_p, []),
@@ -284,17 +285,36 @@ def run_mla(p: Plan, q_nope, q_pe, ckv_cache, kpe_cache, o=None, lse=None, strea
     return o, lse
 
 
-def merge_state(o_a, lse_a, o_b, lse_b, stream=None):
-    """``pkv_merge_state`` on fp32 states ``[rows, dim]`` / ``[rows]``."""
+def merge_state(o_a, lse_a, o_b, lse_b, stream=None, out=None):
+    """``pkv_merge_state`` (fp32 O) or ``pkv_merge_state_bf16`` (bf16 O) on states
+    ``[rows, dim]`` / ``[rows]`` (fp32 LSE, base 2). ``out``: optional ``(o, lse)``
+    to write into (may be the first state)."""
     import torch
-    for t, n in ((o_a, "o_a"), (lse_a, "lse_a"), (o_b, "o_b"), (lse_b, "lse_b")):
+    dt = o_a.dtype
+    if dt not in (torch.float32, torch.bfloat16):
+        raise ValueError("o_a must be float32 or bfloat16")
+    for t, n in ((o_a, "o_a"), (o_b, "o_b")):
+        _check_tensor(t, n, dt)
+    for t, n in ((lse_a, "lse_a"), (lse_b, "lse_b")):
         _check_tensor(t, n, torch.float32)
-    rows, dim = o_a.shape[0], o_a.shape[-1]
-    o = torch.empty_like(o_a)
-    lse = torch.empty_like(lse_a)
-    _check(load_library().pkv_merge_state(o_a.data_ptr(), lse_a.data_ptr(), o_b.data_ptr(), lse_b.data_ptr(),
-                                          o.data_ptr(), lse.data_ptr(), rows, dim, _stream_ptr(stream)))
+    dim = o_a.shape[-1]
+    rows = o_a.numel() // dim
+    o, lse = out if out is not None else (torch.empty_like(o_a), torch.empty_like(lse_a))
+    fn = load_library().pkv_merge_state if dt == torch.float32 else load_library().pkv_merge_state_bf16
+    _check(fn(o_a.data_ptr(), lse_a.data_ptr(), o_b.data_ptr(), lse_b.data_ptr(), o.data_ptr(), lse.data_ptr(), rows,
+              dim, _stream_ptr(stream)))
     return o, lse
+
+
+def cascade_run(prefix_plan: "Plan", suffix_plan: "Plan", q, k_cache, v_cache, stream=None):
+    """Two-level cascade attention (documentation, flashinfer.cascade, "Cascade
+    Attention"): ``prefix_plan`` runs every query against the KV prefix the batch
+    shares (planned non-causal, typically as one request holding all queries),
+    ``suffix_plan`` runs each request against its own pages; the two states are
+    merged by their LSE. Returns ``(o bf16, lse fp32)`` as ``run`` does."""
+    o, lse = run(prefix_plan, q, k_cache, v_cache, stream=stream)
+    o2, lse2 = run(suffix_plan, q, k_cache, v_cache, stream=stream)
+    return merge_state(o, lse, o2, lse2, stream=stream, out=(o, lse))
 
 
 def append_kv(k_new, v_new, append_indptr, kv_indptr, kv_indices, kv_last_page_len, k_cache, v_cache,

@@ -24,6 +24,8 @@ cudaError_t launch_merge_tasks(const LaunchGeom&, const DeviceView&, void*, floa
 cudaError_t launch_merge_state(const float*, const float*, const float*, const float*, float*, float*, int, int,
                                cudaStream_t);
 cudaError_t launch_merge_states(const float*, const float*, int, int, int, void*, float*, cudaStream_t);
+cudaError_t launch_merge_state_bf16(const void*, const float*, const void*, const float*, void*, float*, int, int,
+                                    cudaStream_t);
 }  // namespace pkv
 
 using namespace pkv;
@@ -238,6 +240,16 @@ pkv_status pkv_merge_state(const float* o_a, const float* lse_a, const float* o_
   cudaError_t e = launch_merge_state(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, dim,
                                      static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("merge_state: ") + cudaGetErrorString(e));
+  return PKV_OK;
+}
+
+pkv_status pkv_merge_state_bf16(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                                void* o_out, float* lse_out, int32_t rows, int32_t dim, void* stream) {
+  if (rows < 0 || dim <= 0 || dim > 1024) return fail(PKV_EINVAL, "rows >= 0 and 0 < dim <= 1024 required");
+  if (rows > 0 && (!o_a || !lse_a || !o_b || !lse_b || !o_out || !lse_out)) return fail(PKV_EINVAL, "NULL pointer");
+  cudaError_t e = launch_merge_state_bf16(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, dim,
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("merge_state_bf16: ") + cudaGetErrorString(e));
   return PKV_OK;
 }
 

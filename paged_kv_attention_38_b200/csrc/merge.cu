@@ -68,9 +68,17 @@ __global__ void __launch_bounds__(kWarps * 32) merge_tasks_kernel(const MergeTas
   }
 }
 
-// Two fp32 states -> fp32 state (may alias the first input).
-__global__ void merge_state_kernel(const float* o_a, const float* lse_a, const float* o_b, const float* lse_b,
-                                   float* o_out, float* lse_out, int rows, int dim) {
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ void store(float* p, float x) { *p = x; }
+__device__ __forceinline__ void store(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+
+// Two states -> one state (may alias the first input): fp32 in and out, or
+// bf16 O in and out (the outputs of two attention runs, as in cascade
+// attention); the LSE is fp32 either way.
+template <typename T>
+__global__ void merge_state_kernel(const T* o_a, const float* lse_a, const T* o_b, const float* lse_b,
+                                   T* o_out, float* lse_out, int rows, int dim) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= rows) return;
   const float la = lse_a[warp], lb = lse_b[warp];
@@ -80,7 +88,7 @@ __global__ void merge_state_kernel(const float* o_a, const float* lse_a, const f
   const float L = wa + wb;
   const float fa = L > 0.f ? wa / L : 0.f, fb = L > 0.f ? wb / L : 0.f;
   const size_t base = (size_t)warp * dim;
-  for (int d = lane; d < dim; d += 32) o_out[base + d] = fa * o_a[base + d] + fb * o_b[base + d];
+  for (int d = lane; d < dim; d += 32) store(o_out + base + d, fa * to_f32(o_a[base + d]) + fb * to_f32(o_b[base + d]));
   __syncwarp();
   if (lane == 0) lse_out[warp] = L > 0.f ? mu + __log2f(L) : -INFINITY;
 }
@@ -119,8 +127,19 @@ cudaError_t launch_merge_state(const float* o_a, const float* lse_a, const float
                                float* o_out, float* lse_out, int rows, int dim, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
   const int warps_per_block = 8;
-  merge_state_kernel<<<(rows + warps_per_block - 1) / warps_per_block, warps_per_block * 32, 0, stream>>>(
+  merge_state_kernel<float><<<(rows + warps_per_block - 1) / warps_per_block, warps_per_block * 32, 0, stream>>>(
       o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, dim);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge_state_bf16(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                                    void* o_out, float* lse_out, int rows, int dim, cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  const int warps_per_block = 8;
+  merge_state_kernel<__nv_bfloat16><<<(rows + warps_per_block - 1) / warps_per_block, warps_per_block * 32, 0,
+                                      stream>>>(static_cast<const __nv_bfloat16*>(o_a), lse_a,
+                                                static_cast<const __nv_bfloat16*>(o_b), lse_b,
+                                                static_cast<__nv_bfloat16*>(o_out), lse_out, rows, dim);
   return cudaGetLastError();
 }
 

@@ -387,3 +387,55 @@ def test_append_kv_reports_rows_without_slot():
     torch.cuda.synchronize()
     assert int(status.item()) == 1
     assert int(k_cache.float().sum().item()) == (2 + 3) * hk * d     # request 0's two rows + request 1's three
+
+
+# --------------------------------------------------------------------------- cascade (shared prefix)
+
+def test_merge_state_bf16_kernel():
+    g = torch.Generator().manual_seed(1)
+    rows, dim = 200, 128
+    oa = torch.randn(rows, dim, generator=g).to(torch.bfloat16)
+    ob = torch.randn(rows, dim, generator=g).to(torch.bfloat16)
+    la = torch.randn(rows, generator=g) * 4
+    lb = torch.randn(rows, generator=g) * 4
+    la[0] = -math.inf
+    la[1] = lb[1] = -math.inf
+    o, l = pkv.merge_state(oa.cuda(), la.cuda(), ob.cuda(), lb.cuda())
+    o_ref, l_ref = oracle.merge_state(oa.float().numpy(), la.numpy(), ob.float().numpy(), lb.numpy())
+    assert_parity(o, l, o_ref, l_ref, what="merge_state bf16")
+
+
+def test_cascade_shared_prefix():
+    """Three requests share a 32-key prefix (two pages) and each has its own
+    suffix, its queries being its last suffix tokens. Prefix pass (all queries,
+    non-causal) + suffix pass (causal) merged by LSE equals attention over
+    each request's full page list, prefix pages first."""
+    ps, hq, hk, d = 16, 8, 2, 128
+    g = np.random.default_rng(5)
+    suffix, qo = np.array([20, 45, 7]), np.array([20, 10, 7])
+    pre_pages = 2
+    suf_pages = (suffix + ps - 1) // ps
+    pool = pre_pages + int(suf_pages.sum()) + 3
+    perm = g.permutation(pool).astype(np.int32)
+    prefix_ids, rest = perm[:pre_pages], perm[pre_pages:]
+    suf_ids = np.split(rest[: int(suf_pages.sum())], np.cumsum(suf_pages)[:-1])
+    k = torch.from_numpy(g.standard_normal((pool, ps, hk, d))).to(torch.bfloat16)
+    v = torch.from_numpy(g.standard_normal((pool, ps, hk, d))).to(torch.bfloat16)
+    total_q = int(qo.sum())
+    q = torch.from_numpy(g.standard_normal((total_q, hq, d))).to(torch.bfloat16)
+    qo_indptr = np.concatenate([[0], np.cumsum(qo)]).astype(np.int32)
+    scale = 1.0 / math.sqrt(d)
+    last_suf = (suffix - (suf_pages - 1) * ps).astype(np.int32)
+    # the oracle: each request's full table = prefix pages + its own pages
+    full_indptr = np.concatenate([[0], np.cumsum(pre_pages + suf_pages)]).astype(np.int32)
+    full_ids = np.concatenate([np.concatenate([prefix_ids, s]) for s in suf_ids]).astype(np.int32)
+    o_ref, l_ref = oracle.paged_attention(q, k, v, qo_indptr, full_indptr, full_ids, last_suf, ps, True, scale)
+    # GPU: prefix pass as one request holding every query, suffix pass per request
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    pre_plan = pkv.plan(np.array([0, total_q], np.int32), np.array([0, pre_pages], np.int32), dev(prefix_ids),
+                        np.array([ps], np.int32), hq, hk, d, ps, False, scale)
+    suf_indptr = np.concatenate([[0], np.cumsum(suf_pages)]).astype(np.int32)
+    suf_plan = pkv.plan(qo_indptr, suf_indptr, dev(np.concatenate(suf_ids)), last_suf, hq, hk, d, ps, True, scale)
+    o, l = pkv.cascade_run(pre_plan, suf_plan, q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    assert_parity(o, l, o_ref, l_ref, what="cascade")

@@ -559,3 +559,36 @@ def test_append_pin_catches_off_by_one(monkeypatch):
             test_append_round_trip_through_gather()
         except IndexError as e:  # a shifted position may also run off the page list
             raise AssertionError(str(e))
+
+
+def test_cascade_identity():
+    """Shared-prefix (cascade) decomposition: a non-causal pass of every query
+    over the shared prefix merged with a causal pass over each request's own
+    pages equals attention over prefix + own pages (queries are the last tokens
+    of their suffix, so the whole prefix is visible to them)."""
+    ps, hq, hk, d = 16, 8, 2, 32
+    g = np.random.default_rng(5)
+    suffix, qo = np.array([20, 45, 7]), np.array([20, 10, 7])
+    pre_pages = 2
+    suf_pages = (suffix + ps - 1) // ps
+    pool = pre_pages + int(suf_pages.sum()) + 3
+    perm = g.permutation(pool).astype(np.int32)
+    prefix_ids, rest = perm[:pre_pages], perm[pre_pages:]
+    suf_ids = np.split(rest[: int(suf_pages.sum())], np.cumsum(suf_pages)[:-1])
+    k = torch.from_numpy(g.standard_normal((pool, ps, hk, d))).to(torch.bfloat16)
+    v = torch.from_numpy(g.standard_normal((pool, ps, hk, d))).to(torch.bfloat16)
+    total_q = int(qo.sum())
+    q = torch.from_numpy(g.standard_normal((total_q, hq, d))).to(torch.bfloat16)
+    qo_indptr = np.concatenate([[0], np.cumsum(qo)]).astype(np.int32)
+    scale = 1 / math.sqrt(d)
+    last_suf = (suffix - (suf_pages - 1) * ps).astype(np.int32)
+    full_indptr = np.concatenate([[0], np.cumsum(pre_pages + suf_pages)]).astype(np.int32)
+    full_ids = np.concatenate([np.concatenate([prefix_ids, s]) for s in suf_ids]).astype(np.int32)
+    o_ref, l_ref = oracle.paged_attention(q, k, v, qo_indptr, full_indptr, full_ids, last_suf, ps, True, scale)
+    o1, l1 = oracle.paged_attention(q, k, v, np.array([0, total_q], np.int32), np.array([0, pre_pages], np.int32),
+                                    prefix_ids, np.array([ps], np.int32), ps, False, scale)
+    suf_indptr = np.concatenate([[0], np.cumsum(suf_pages)]).astype(np.int32)
+    o2, l2 = oracle.paged_attention(q, k, v, qo_indptr, suf_indptr, np.concatenate(suf_ids), last_suf, ps, True,
+                                    scale)
+    o, lse = oracle.merge_state(o1, l1, o2, l2)
+    assert np.abs(o - o_ref).max() < 1e-12 and np.abs(lse - l_ref).max() < 1e-12
