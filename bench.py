@@ -242,6 +242,35 @@ class Case:
             pkv.run(self.plan, self.q, self.k, self.v, self.o, self.lse)
 
 
+class AppendCase:
+    """Paged KV append of a whole prefill batch: every request's rows written into
+    its pages (the table after the append), K and V, resident in HBM."""
+
+    def __init__(self, p: W.PagedProblem, device):
+        self.p = p
+        self.k, self.v = p.k_cache.to(device), p.v_cache.to(device)
+        kv = p.kv_lens
+        self.nnz = int(kv.sum())
+        gen = torch.Generator().manual_seed(p.seed + 500)
+        shape = (self.nnz, p.num_kv_heads, p.head_dim)
+        self.k_new = torch.randn(shape, generator=gen).to(torch.bfloat16).to(device)
+        self.v_new = torch.randn(shape, generator=gen).to(torch.bfloat16).to(device)
+        dev = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.int32)).to(device)
+        self.append_indptr = dev(np.concatenate([[0], np.cumsum(kv)]))
+        self.kv_indptr, self.kv_indices, self.last = dev(p.kv_indptr), dev(p.kv_indices), dev(p.kv_last_page_len)
+        self.launches = 1
+
+    @property
+    def bytes(self) -> float:
+        """New K and V rows read once and written once, plus the index arrays."""
+        rows = 2 * 2 * self.nnz * self.p.num_kv_heads * self.p.head_dim
+        return float(2 * rows + 4 * (len(self.p.kv_indices) + 3 * (self.p.batch + 1)))
+
+    def run(self):
+        pkv.append_kv(self.k_new, self.v_new, self.append_indptr, self.kv_indptr, self.kv_indices, self.last,
+                      self.k, self.v)
+
+
 def time_case(case: Case, flush: torch.Tensor, steps: int, warmup: int):
     """Median and mean kernel time (ms) of `case.run`, L2 flushed before every launch."""
     for _ in range(warmup):
@@ -427,6 +456,16 @@ def run_ours(args):
     job_bytes_s, dec_ms = job_throughput(dec_bytes, mean_ms(dec), world)
     mla_ms = max_over_ranks(mean_ms(mla), world) if mla else None
     step_ms = pre_ms + dec_ms + (mla_ms or 0.0)
+
+    # Rows beyond the step (timed the same way, each alone between L2 flushes):
+    # MLA decode and the paged KV append.
+    extra_steps = max(3, min(args.steps, 20))
+    mdec = Case(W.mla_decode(shard=rank), device)
+    mdec_med, mdec_ms_local = time_case(mdec, flush, extra_steps, 3)
+    mdec_ms = max_over_ranks(mdec_ms_local, world)
+    app = AppendCase(W.gqa_prefill(shard=rank), device)
+    app_med, app_ms_local = time_case(app, flush, extra_steps, 3)
+    app_ms = max_over_ranks(app_ms_local, world)
     tflops = job_flops_s / 1e12
     per_gpu_tflops = pre_flops / (pre_ms * 1e-3) / 1e12
     dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
@@ -456,7 +495,15 @@ def run_ours(args):
             "bound": "tensor", "achieved": round(mla_tf, 2), "peak": peak_burst, "unit": "TFLOP/s",
             "frac": round(mla_tf / peak_burst, 4),
             "traffic": profiled_traffic("mla_h16_ckv512_kpe64_ps1.md", MLA_SOURCES), "ms": round(mla_ms, 4)}
-    dominant = max(roofs, key=lambda k: roofs[k]["ms"])
+    mdec_gbs = decode_bytes(mdec.p) / (mdec_ms * 1e-3) / 1e9
+    roofs["mla_decode_kernel (b64/h16/ckv512/kpe64/ps1)"] = {
+        "bound": "hbm", "achieved": round(mdec_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(mdec_gbs / hbm, 4),
+        "traffic": None, "ms": round(mdec_ms, 4), "in_step": False}
+    app_gbs = app.bytes / (app_ms * 1e-3) / 1e9
+    roofs["append_kernel (h16/kv1/d128/ps64 batch)"] = {
+        "bound": "hbm", "achieved": round(app_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(app_gbs / hbm, 4),
+        "traffic": None, "ms": round(app_ms, 4), "in_step": False}
+    dominant = max((k for k in roofs if roofs[k].get("in_step", True)), key=lambda k: roofs[k]["ms"])
     roofline = dict(roofs[dominant], kernel=dominant,
                     peak_kind=f"{peak_kind} (burst bf16 for tensor-bound kernels timed alone between L2 flushes; "
                               "copy bandwidth for HBM-bound)")
@@ -504,6 +551,13 @@ def run_ours(args):
         line["mla"] = {"value": round(mla_flops / (mla_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                        "ms": round(mla_ms, 4), "flops": mla_flops,
                        "workload": "mla_paged_prefill_causal_h16_ckv512_kpe64_ps1, batch 4, U[256,2048]"}
+    line["mla_decode"] = {"value": round(mdec_gbs, 1), "unit": "GB/s", "ms": round(mdec_ms, 4),
+                          "bytes": decode_bytes(mdec.p), "units": mdec.plan.num_units, "merges": mdec.plan.num_merges,
+                          "workload": "mla_paged_decode_h16_ckv512_kpe64_ps1, batch 64, kv_len U[1024,8192]",
+                          "timed": "alone, outside the step, L2 flushed before each launch"}
+    line["append"] = {"value": round(app_gbs, 1), "unit": "GB/s", "ms": round(app_ms, 4), "bytes": app.bytes,
+                      "rows": app.nnz, "workload": "append of the whole h16/kv1/d128/ps64 prefill batch (K and V)",
+                      "timed": "alone, outside the step, L2 flushed before each launch"}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if args.sweep:
@@ -518,6 +572,14 @@ def run_only(args, device, flush):
               "sparse": lambda: W.sparse_vs_dense(16, 2048, False),
               "dense": lambda: W.sparse_vs_dense(16, 2048, True),
               "mla_decode": W.mla_decode}
+    if args.only == "append":
+        c = AppendCase(W.gqa_prefill(), device)
+        sampler = ClockSampler(device.index or 0)
+        with sampler:
+            med, mean = time_case(c, flush, args.steps, args.warmup)
+        print(json.dumps({"only": "append", "ms_median": med, "ms_mean": mean, "gbs": c.bytes / (med * 1e-3) / 1e9,
+                          "rows": c.nnz, "clocks": sampler.summary()}), flush=True)
+        return
     c = Case(makers[args.only](), device)
     sampler = ClockSampler(device.index or 0)
     with sampler:
@@ -586,7 +648,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--sweep", action="store_true", help="also run the vector-sparse vs dense sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "decode_small", "mla", "mla_decode", "sparse", "dense"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "decode_small", "mla", "mla_decode", "sparse", "dense", "append"], default=None,
                     help="time one workload alone (profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
