@@ -7,7 +7,9 @@
 // The split-KV schedule (discussion #15, disable_split_kv) relies on it.
 //
 // One warp per output row: each lane reads every part's LSE (a handful of
-// floats), then strides over the row's columns. The reads are coalesced along
+// floats), then strides over the row's columns. A task's rows are spread over
+// blockIdx.y as well, so a few tasks with many rows (MLA decode: 16 heads x 512
+// columns x tens of parts) still fill the GPU. The reads are coalesced along
 // the row; the data is read once, so the kernel is bound by HBM traffic of
 // the partials (tiny next to the KV stream that produced them).
 #include <cuda_bf16.h>
@@ -20,7 +22,7 @@ namespace pkv {
 
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 4;
 
 __device__ __forceinline__ float part_max(const float* lse, size_t stride, int num) {
   float m = -INFINITY;
@@ -40,7 +42,7 @@ __global__ void __launch_bounds__(kWarps * 32) merge_tasks_kernel(const MergeTas
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Dv = g.head_dim_v, G = g.group, R = g.part_rows;
   const size_t slot_stride = (size_t)R;
-  for (int r = warp; r < t.rows; r += kWarps) {
+  for (int r = blockIdx.y * kWarps + warp; r < t.rows; r += gridDim.y * kWarps) {
     const float* lp = part_lse + (size_t)t.slot0 * R + r;
     const float m = part_max(lp, slot_stride, t.num);
     const float mu = m == -INFINITY ? 0.f : m;
@@ -118,8 +120,9 @@ __global__ void merge_states_kernel(const float* o_parts, const float* lse_parts
 cudaError_t launch_merge_tasks(const LaunchGeom& g, const DeviceView& dv, void* o, float* lse,
                                cudaStream_t stream) {
   if (g.num_merge == 0) return cudaSuccess;
-  merge_tasks_kernel<<<g.num_merge, kWarps * 32, 0, stream>>>(dv.merges, g, dv.reqs, dv.part_o, dv.part_lse,
-                                                              static_cast<__nv_bfloat16*>(o), lse);
+  const dim3 grid(g.num_merge, (g.part_rows + kWarps - 1) / kWarps);
+  merge_tasks_kernel<<<grid, kWarps * 32, 0, stream>>>(dv.merges, g, dv.reqs, dv.part_o, dv.part_lse,
+                                                       static_cast<__nv_bfloat16*>(o), lse);
   return cudaGetLastError();
 }
 
