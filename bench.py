@@ -91,8 +91,10 @@ def decode_bytes(p: W.PagedProblem) -> float:
 # ----------------------------------------------------------------- profile figures
 
 PREFILL_SOURCES = ("prefill_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
-DECODE_SOURCES = ("decode_sm100.cu", "merge.cu", "sm100_ptx.cuh", "pkv_internal.h")
+DECODE_SOURCES = ("decode_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
 MLA_SOURCES = ("mla_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
+MLA_DECODE_SOURCES = ("mla_decode_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
+APPEND_SOURCES = ("append.cu",)
 
 
 def kernel_source_sha(files) -> str:
@@ -498,11 +500,13 @@ def run_ours(args):
     mdec_gbs = decode_bytes(mdec.p) / (mdec_ms * 1e-3) / 1e9
     roofs["mla_decode_kernel (b64/h16/ckv512/kpe64/ps1)"] = {
         "bound": "hbm", "achieved": round(mdec_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(mdec_gbs / hbm, 4),
-        "traffic": None, "ms": round(mdec_ms, 4), "in_step": False}
+        "traffic": profiled_traffic("mla_decode_b64_h16_ckv512_kpe64_ps1.md", MLA_DECODE_SOURCES), "ms": round(mdec_ms, 4),
+        "in_step": False}
     app_gbs = app.bytes / (app_ms * 1e-3) / 1e9
     roofs["append_kernel (h16/kv1/d128/ps64 batch)"] = {
         "bound": "hbm", "achieved": round(app_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(app_gbs / hbm, 4),
-        "traffic": None, "ms": round(app_ms, 4), "in_step": False}
+        "traffic": profiled_traffic("append_h16_kv1_d128_ps64.md", APPEND_SOURCES), "ms": round(app_ms, 4),
+        "in_step": False}
     dominant = max((k for k in roofs if roofs[k].get("in_step", True)), key=lambda k: roofs[k]["ms"])
     roofline = dict(roofs[dominant], kernel=dominant,
                     peak_kind=f"{peak_kind} (burst bf16 for tensor-bound kernels timed alone between L2 flushes; "
