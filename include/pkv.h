@@ -93,7 +93,10 @@ typedef struct pkv_plan_options {
   int32_t num_sms;          /* SMs to schedule for; 0 = query the current device */
   int32_t disable_split_kv; /* 1 = never split a request's KV across CTAs */
   int32_t kv_chunk;         /* >0: force this KV chunk length (tokens) when splitting; 0 = auto */
-  int32_t reserved[5];
+  int32_t kv_layout;        /* GQA/MHA page layout (FlashInfer 0.7.4 documentation, "KV-Cache Layout in
+                               FlashInfer", "Layout: NHD/HND"): 0 = NHD, a page is [page_size, Hk, D];
+                               1 = HND, a page is [Hk, page_size, D]. MLA pools have no head axis: ignored. */
+  int32_t reserved[4];
 } pkv_plan_options;
 
 /* Plan a batch: builds the CTA work list on the host.
@@ -172,8 +175,10 @@ PKV_API pkv_status pkv_merge_states(const float* o_parts, const float* lse_parts
  * kv_indices[kv_indptr[b] + pos / page_size], slot pos % page_size.
  * k_new [nnz, num_kv_heads, head_dim], v_new [nnz, num_kv_heads, head_dim_v]:
  * DEVICE bf16 (any 2-byte type: bytes are copied unchanged). k_cache
- * [num_pages, page_size, num_kv_heads, head_dim], v_cache likewise with
- * head_dim_v: DEVICE, updated in place; every other slot is left untouched.
+ * [num_pages, page_size, num_kv_heads, head_dim] (kv_layout 0, NHD) or
+ * [num_pages, num_kv_heads, page_size, head_dim] (kv_layout 1, HND), v_cache
+ * likewise with head_dim_v: DEVICE, updated in place; every other slot is left
+ * untouched.
  * MLA caches fit the same call with num_kv_heads 1: k = ckv (512), v = kpe (64).
  * Head dims must be multiples of 8 and pointers 16-byte aligned.
  * A row whose position falls outside its request, or whose page id is not in
@@ -183,7 +188,7 @@ PKV_API pkv_status pkv_append_kv(const void* k_new, const void* v_new, const int
                                  const int32_t* kv_indptr, const int32_t* kv_indices,
                                  const int32_t* kv_last_page_len, int32_t batch, int32_t num_kv_heads,
                                  int32_t head_dim, int32_t head_dim_v, int32_t page_size, int32_t num_pages,
-                                 void* k_cache, void* v_cache, int32_t* status, void* stream);
+                                 int32_t kv_layout, void* k_cache, void* v_cache, int32_t* status, void* stream);
 
 /* Paged decode (one query token per request) for callers that cannot allocate
  * device memory: code under an allocator that forbids new device allocations

@@ -43,7 +43,7 @@ class PkvError(RuntimeError):
 
 class _Options(ctypes.Structure):
     _fields_ = [("num_sms", ctypes.c_int32), ("disable_split_kv", ctypes.c_int32),
-                ("kv_chunk", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5)]
+                ("kv_chunk", ctypes.c_int32), ("kv_layout", ctypes.c_int32), ("reserved", ctypes.c_int32 * 4)]
 
 
 _lib = None
@@ -69,7 +69,7 @@ _SIGS = {
     "pkv_plan_merge_tasks": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
     "pkv_plan_cta_units": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
     "pkv_merge_state_bf16": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
-    "pkv_append_kv": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P, _P, _P] + [ctypes.c_int32] * 6 + [_P, _P, _P, _P]),
+    "pkv_append_kv": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P, _P, _P] + [ctypes.c_int32] * 7 + [_P, _P, _P, _P]),
     "pkv_plan_destroy": (None, [_P]),
     "pkv_last_error": (ctypes.c_char_p, []),
     "pkv_version": (ctypes.c_char_p, []),
@@ -194,25 +194,27 @@ class Plan:
             _lib.pkv_plan_destroy(h)
 
 
-def _options(num_sms, disable_split_kv, kv_chunk):
+def _options(num_sms, disable_split_kv, kv_chunk, kv_layout=0):
     o = _Options()
     o.num_sms, o.disable_split_kv, o.kv_chunk = int(num_sms), int(bool(disable_split_kv)), int(kv_chunk)
+    o.kv_layout = int(kv_layout)
     return o
 
 
 def plan(qo_indptr, kv_indptr, kv_indices, kv_last_page_len, num_qo_heads, num_kv_heads, head_dim,
          page_size, causal, sm_scale, *, num_sms: int = 0, disable_split_kv: bool = False,
-         kv_chunk: int = 0, upload: bool = True, device=None, stream=None) -> Plan:
+         kv_chunk: int = 0, kv_layout: int = 0, upload: bool = True, device=None, stream=None) -> Plan:
     """Plan a GQA/MHA paged-attention batch (``pkv_plan_create`` + ``pkv_plan_upload``).
 
     ``qo_indptr``, ``kv_indptr``, ``kv_last_page_len`` are host int32 arrays;
     ``kv_indices`` is a device int32 tensor (may be None with ``upload=False``
-    to inspect the schedule on a machine without a GPU).
+    to inspect the schedule on a machine without a GPU). ``kv_layout``: 0 NHD
+    pools ``[num_pages, page_size, Hk, D]``, 1 HND ``[num_pages, Hk, page_size, D]``.
     """
     lib = load_library()
     qo, kv, last = _host_i32(qo_indptr), _host_i32(kv_indptr), _host_i32(kv_last_page_len)
     h = _P()
-    opts = _options(num_sms, disable_split_kv, kv_chunk)
+    opts = _options(num_sms, disable_split_kv, kv_chunk, kv_layout)
     _check(lib.pkv_plan_create(_i32p(qo), _i32p(kv), _ptr(kv_indices), _i32p(last), len(last), num_qo_heads,
                                num_kv_heads, head_dim, page_size, int(bool(causal)), float(sm_scale),
                                ctypes.byref(opts), ctypes.byref(h)))
@@ -318,11 +320,12 @@ def cascade_run(prefix_plan: "Plan", suffix_plan: "Plan", q, k_cache, v_cache, s
 
 
 def append_kv(k_new, v_new, append_indptr, kv_indptr, kv_indices, kv_last_page_len, k_cache, v_cache,
-              status=None, stream=None):
+              status=None, stream=None, kv_layout: int = 0):
     """``pkv_append_kv``: write new rows ``k_new`` / ``v_new`` ``[nnz, Hk, D]`` into the
     page pools ``[num_pages, page_size, Hk, D]`` in place, at the last positions of
     each request under the page table after the append (all index arrays int32 on
-    the device). ``status``: optional int32 device tensor set to 1 on a bad row."""
+    the device). ``kv_layout`` 1: pools are HND ``[num_pages, Hk, page_size, D]``.
+    ``status``: optional int32 device tensor set to 1 on a bad row."""
     import torch
     for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
         _check_tensor(t, n)
@@ -335,10 +338,12 @@ def append_kv(k_new, v_new, append_indptr, kv_indptr, kv_indices, kv_last_page_l
         k_cache, v_cache = k_cache.unsqueeze(2), v_cache.unsqueeze(2)
         k_new, v_new = k_new.reshape(k_new.shape[0], 1, -1), v_new.reshape(v_new.shape[0], 1, -1)
     num_pages, page_size, hk, d = k_cache.shape
+    if kv_layout == 1:
+        num_pages, hk, page_size, d = k_cache.shape
     _check(load_library().pkv_append_kv(
         k_new.data_ptr(), v_new.data_ptr(), append_indptr.data_ptr(), int(k_new.shape[0]), kv_indptr.data_ptr(),
         kv_indices.data_ptr(), kv_last_page_len.data_ptr(), int(kv_last_page_len.shape[0]), hk, d,
-        int(v_cache.shape[-1]), page_size, num_pages, k_cache.data_ptr(), v_cache.data_ptr(),
+        int(v_cache.shape[-1]), page_size, num_pages, int(kv_layout), k_cache.data_ptr(), v_cache.data_ptr(),
         status.data_ptr() if status is not None else None, _stream_ptr(stream)))
 
 

@@ -33,10 +33,11 @@ struct AppendArgs {
   const int32_t* kv_indptr;
   const int32_t* kv_indices;
   const int32_t* kv_last_page_len;
-  uint4* k_cache;      // [num_pages, P, Hk, Dk]
-  uint4* v_cache;      // [num_pages, P, Hk, Dv]
+  uint4* k_cache;      // [num_pages, P, Hk, Dk] (NHD) or [num_pages, Hk, P, Dk] (HND)
+  uint4* v_cache;      // likewise with Dv
   int32_t* status;     // optional: set to 1 when a row had no valid slot
   int32_t batch, num_kv_heads, chunks_k, chunks_v, page_size, num_pages;
+  int32_t hnd;         // pages laid out [kv head][slot][D] instead of [slot][kv head][D]
   int64_t nnz;
 };
 
@@ -69,7 +70,8 @@ __global__ void __launch_bounds__(kThreads) append_kernel(const AppendArgs a) {
       if (a.status) atomicExch(a.status, 1);
       continue;
     }
-    const int64_t slot_row = ((int64_t)page * a.page_size + pos % a.page_size) * a.num_kv_heads + h;
+    const int64_t slot_row = a.hnd ? ((int64_t)page * a.num_kv_heads + h) * a.page_size + pos % a.page_size
+                                   : ((int64_t)page * a.page_size + pos % a.page_size) * a.num_kv_heads + h;
     const int64_t new_row = t * a.num_kv_heads + h;
     if (c < a.chunks_k) a.k_cache[slot_row * a.chunks_k + c] = a.k_new[new_row * a.chunks_k + c];
     if (c < a.chunks_v) a.v_cache[slot_row * a.chunks_v + c] = a.v_new[new_row * a.chunks_v + c];
@@ -85,7 +87,7 @@ extern "C" pkv_status pkv_append_kv(const void* k_new, const void* v_new, const 
                                     const int32_t* kv_indptr, const int32_t* kv_indices,
                                     const int32_t* kv_last_page_len, int32_t batch, int32_t num_kv_heads,
                                     int32_t head_dim, int32_t head_dim_v, int32_t page_size, int32_t num_pages,
-                                    void* k_cache, void* v_cache, int32_t* status, void* stream) {
+                                    int32_t kv_layout, void* k_cache, void* v_cache, int32_t* status, void* stream) {
   using namespace pkv;
   if (batch < 0 || nnz < 0) {
     set_last_error("batch and nnz must be non-negative");
@@ -95,6 +97,10 @@ extern "C" pkv_status pkv_append_kv(const void* k_new, const void* v_new, const 
   if (num_kv_heads <= 0 || head_dim <= 0 || head_dim_v <= 0 || head_dim % 8 != 0 || head_dim_v % 8 != 0) {
     set_last_error("num_kv_heads > 0 and head dims that are positive multiples of 8 required");
     return PKV_EUNSUPPORTED;
+  }
+  if (kv_layout != 0 && kv_layout != 1) {
+    set_last_error("kv_layout must be 0 (NHD) or 1 (HND)");
+    return PKV_EINVAL;
   }
   if (page_size <= 0 || num_pages <= 0) {
     set_last_error("page_size and num_pages must be positive");
@@ -126,6 +132,7 @@ extern "C" pkv_status pkv_append_kv(const void* k_new, const void* v_new, const 
   a.page_size = page_size;
   a.num_pages = num_pages;
   a.nnz = nnz;
+  a.hnd = kv_layout;
   const int64_t total = nnz * num_kv_heads * (a.chunks_k > a.chunks_v ? a.chunks_k : a.chunks_v);
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {

@@ -67,7 +67,8 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int D>
+// kHnd: pages laid out [kv head][slot][D] (HND) instead of [slot][kv head][D].
+template <int D, bool kHnd>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_constant__ Args a) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kTileBytes = kTile * D * 2;
@@ -99,7 +100,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
       const int r = c / kChunks, ch = c % kChunks;
       const int pos = unit.kv_lo + j * kTile + r;
       const bool ok = page[i] >= 0;
-      const size_t off = ok ? (((size_t)page[i] * P + (pos & (P - 1))) * Hk + unit.kv_head) * D + ch * 8 : 0;
+      size_t off = 0;
+      if constexpr (kHnd)
+        off = ok ? (((size_t)page[i] * Hk + unit.kv_head) * P + (pos & (P - 1))) * D + ch * 8 : 0;
+      else
+        off = ok ? (((size_t)page[i] * P + (pos & (P - 1))) * Hk + unit.kv_head) * D + ch * 8 : 0;
       cp_async_16(kdst + kv_off<D>(r, ch), a.k + off, ok ? 16u : 0u);
       cp_async_16(vdst + kv_off<D>(r, ch), a.v + off, ok ? 16u : 0u);
     }
@@ -269,12 +274,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_consta
   }
 }
 
-template <int D>
+template <int D, bool kHnd>
 cudaError_t launch(const Args& a, cudaStream_t stream) {
   const size_t pipe = (size_t)kStages * 2 * kTile * D * 2;
   const size_t comb = (size_t)4 * 16 * D * 4 + 2 * 4 * 16 * 4;
   const size_t smem = pipe > comb ? pipe : comb;
-  auto kern = decode_kernel<D>;
+  auto kern = decode_kernel<D, kHnd>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   // all of the unified L1 / shared array as shared memory, so two CTAs fit per SM
   if (e == cudaSuccess)
@@ -291,8 +296,9 @@ cudaError_t launch_decode(const LaunchGeom& g, const DeviceView& dv, const int32
   if (g.num_units == 0) return cudaSuccess;
   Args a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
          static_cast<const __nv_bfloat16*>(v), kv_indices, static_cast<__nv_bfloat16*>(o), lse, g, dv};
-  if (g.head_dim == 128) return launch<128>(a, stream);
-  if (g.head_dim == 64) return launch<64>(a, stream);
+  const bool hnd = g.kv_layout == 1;
+  if (g.head_dim == 128) return hnd ? launch<128, true>(a, stream) : launch<128, false>(a, stream);
+  if (g.head_dim == 64) return hnd ? launch<64, true>(a, stream) : launch<64, false>(a, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -72,6 +72,7 @@ struct LaunchGeom {
   int32_t num_merge;
   int32_t total_q;        // rows of q (tokens)
   int32_t num_ctas;       // CTAs of the main launch (prefill: persistent, one unit list each)
+  int32_t kv_layout;      // 0 NHD [page, slot, kv head, D]; 1 HND [page, kv head, slot, D]
 };
 
 // Device pointers into the workspace after upload.

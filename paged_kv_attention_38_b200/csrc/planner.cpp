@@ -50,6 +50,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   }
   if (in.num_qo_heads <= 0 || in.num_kv_heads <= 0) { *err = "head counts must be positive"; return 1; }
   if (in.num_qo_heads % in.num_kv_heads != 0) { *err = "num_qo_heads % num_kv_heads != 0"; return 1; }
+  if (in.kv_layout != 0 && in.kv_layout != 1) { *err = "kv_layout must be 0 (NHD) or 1 (HND)"; return 1; }
   if (!is_pow2(in.page_size) || in.page_size > 256) {
     *err = "page_size must be a power of two in [1, 256]"; return 2;
   }
@@ -257,6 +258,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   gm.num_merge = (int32_t)s.merges.size();
   gm.total_q = in.batch > 0 ? in.qo_indptr[in.batch] : 0;
   gm.num_ctas = num_ctas;
+  gm.kv_layout = mla ? 0 : in.kv_layout;  // a latent pool has no head axis: both layouts coincide
   *out = std::move(s);
   return 0;
 }

@@ -32,6 +32,7 @@ struct PlanInput {
   int32_t num_sms;
   int32_t disable_split_kv;
   int32_t kv_chunk;     // > 0 forces the split chunk
+  int32_t kv_layout;    // 0 NHD, 1 HND (GQA/MHA pools)
 };
 
 struct Schedule {

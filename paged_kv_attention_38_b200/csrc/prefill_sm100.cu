@@ -118,7 +118,7 @@ struct Args {
 // units with keys), so the producer streams the next unit's Q and K/V and the
 // tensor core starts its first QK^T while the softmax warps still write the
 // previous unit's output.
-template <int D, bool kRows>
+template <int D, bool kRows, bool kHnd>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Args a) {
   extern __shared__ uint8_t smem_raw[];
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -232,6 +232,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             mbar_arrive_expect_tx(&sm.full[slot], kBlockN * D * 2);
             const CUtensorMap* tm = is_v ? &a.tm_v : &a.tm_k;
             const uint32_t dst = smem_u32(sm.kv[slot]);
+            if constexpr (kHnd) {
+              // HND view [page x kv head][slot][D]: one kv head's slots of a page are contiguous
+              if (P >= kBlockN) {
+                const int ph = __ldg(a.kv_indices + req.page0 + (pos0 >> shift)) * Hk + unit.kv_head;
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h)
+                  tma_load_3d(dst + h * (kTileM * 128), tm, &sm.full[slot], h * 64, pos0 & (P - 1), ph);
+              } else {
+                const int npc = kBlockN >> shift;
+                const int lp0 = pos0 >> shift;
+                for (int pi = 0; pi < npc; ++pi) {
+                  const int lp = lp0 + pi;
+                  const int ph = lp < n_pages_req ? __ldg(a.kv_indices + req.page0 + lp) * Hk + unit.kv_head : a.oob_row;
+#pragma unroll
+                  for (int h = 0; h < D / 64; ++h)
+                    tma_load_3d(dst + h * (kTileM * 128) + pi * P * 128, tm, &sm.full[slot], h * 64, 0, ph);
+                }
+              }
+            } else {
             if (P >= kBlockN) {
               const int page = __ldg(a.kv_indices + req.page0 + (pos0 >> shift));
               const int row = page * P + (pos0 & (P - 1));
@@ -247,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 for (int h = 0; h < D / 64; ++h)
                   tma_load_3d(dst + h * (kTileM * 128) + pi * P * 128, tm, &sm.full[slot], h * 64, unit.kv_head, row);
               }
+            }
             }
           }
         } else {
@@ -272,7 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             const size_t row_stride = (size_t)Hk * D;
             for (int r = pt / kChunks; r < kBlockN; r += kRowStep) {
               const int src = sm.rowsrc[r];
-              const __nv_bfloat16* g = src >= 0 ? base + (size_t)src * row_stride + ch * 8 : a.k;
+              const __nv_bfloat16* g = a.k;
+              if constexpr (kHnd) {  // page src / P, slot src % P, [page][kv head][slot][D]
+                if (src >= 0)
+                  g = (is_v ? a.v : a.k) + (((size_t)(src >> shift) * Hk + unit.kv_head) * P + (src & (P - 1))) * D + ch * 8;
+              } else {
+                if (src >= 0) g = base + (size_t)src * row_stride + ch * 8;
+              }
               cp_async_16(dst + r * 128 + (col_off ^ ((r & 7) << 4)), g, src >= 0 ? 16u : 0u);
             }
           } else {
@@ -283,7 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             for (int c = pt; c < kBlockN * kChunks; c += kProdThreads) {
               const int r = c / kChunks, ch = c % kChunks;
               const int src = sm.rowsrc[r];
-              const __nv_bfloat16* g = src >= 0 ? base + ((size_t)src * Hk + unit.kv_head) * D + ch * 8 : base;
+              const __nv_bfloat16* g;
+              if constexpr (kHnd)
+                g = src >= 0 ? base + (((size_t)(src >> shift) * Hk + unit.kv_head) * P + (src & (P - 1))) * D + ch * 8
+                             : base;
+              else
+                g = src >= 0 ? base + ((size_t)src * Hk + unit.kv_head) * D + ch * 8 : base;
               cp_async_16(dst + tile_off(r, ch), g, src >= 0 ? 16u : 0u);
             }
           }
@@ -662,23 +693,27 @@ bool make_map(CUtensorMap* m, const void* base, int D, int heads, int64_t rows, 
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool kRows>
+template <int D, bool kRows, bool kHnd>
 cudaError_t launch_as(const Args& a, cudaStream_t stream) {
   const size_t smem = sizeof(Smem<D>) + 1024;
   static bool configured = false;
   if (!configured) {
     cudaError_t e =
-        cudaFuncSetAttribute(prefill_kernel<D, kRows>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(prefill_kernel<D, kRows, kHnd>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  prefill_kernel<D, kRows><<<a.g.num_ctas, kThreads, smem, stream>>>(a);
+  prefill_kernel<D, kRows, kHnd><<<a.g.num_ctas, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
+// One instance per K/V path and page layout, so that each holds only its own
+// address arithmetic (the NHD instances are unchanged by the HND ones).
 template <int D>
 cudaError_t launch(const Args& a, cudaStream_t stream) {
-  return a.kv_tma ? launch_as<D, false>(a, stream) : launch_as<D, true>(a, stream);
+  if (a.g.kv_layout == 1)
+    return a.kv_tma ? launch_as<D, false, true>(a, stream) : launch_as<D, true, true>(a, stream);
+  return a.kv_tma ? launch_as<D, false, false>(a, stream) : launch_as<D, true, false>(a, stream);
 }
 
 }  // namespace
@@ -697,12 +732,21 @@ cudaError_t launch_prefill(const LaunchGeom& g, const DeviceView& dv, const int3
   a.g = g;
   a.dv = dv;
   const int64_t pool_rows = (int64_t)num_pages * g.page_size;
-  a.oob_row = (int32_t)pool_rows;
+  const bool hnd = g.kv_layout == 1;
+  // K/V tensor-map rows: NHD pool rows (slots), HND (page, kv head) pairs
+  const int64_t map_rows = hnd ? (int64_t)num_pages * g.num_kv_heads : pool_rows;
+  a.oob_row = (int32_t)std::min<int64_t>(map_rows, INT32_MAX);
   a.q_tma = (kTileM % g.group == 0) &&
             make_map(&a.tm_q, q, g.head_dim, g.num_qo_heads, g.total_q, g.group, kTileM / g.group);
-  a.kv_tma = g.page_size >= 8 && pool_rows < INT32_MAX &&
-             make_map(&a.tm_k, k, g.head_dim, g.num_kv_heads, pool_rows, 1, g.page_size < kBlockN ? g.page_size : kBlockN) &&
-             make_map(&a.tm_v, v, g.head_dim, g.num_kv_heads, pool_rows, 1, g.page_size < kBlockN ? g.page_size : kBlockN);
+  const int box = g.page_size < kBlockN ? g.page_size : kBlockN;
+  if (hnd)  // [page x kv head][slot][D]: dims {D, page_size, pages x heads}, box {64, slots, 1}
+    a.kv_tma = g.page_size >= 8 && map_rows < INT32_MAX &&
+               make_map(&a.tm_k, k, g.head_dim, g.page_size, map_rows, box, 1) &&
+               make_map(&a.tm_v, v, g.head_dim, g.page_size, map_rows, box, 1);
+  else
+    a.kv_tma = g.page_size >= 8 && pool_rows < INT32_MAX &&
+               make_map(&a.tm_k, k, g.head_dim, g.num_kv_heads, pool_rows, 1, box) &&
+               make_map(&a.tm_v, v, g.head_dim, g.num_kv_heads, pool_rows, 1, box);
   if (g.head_dim == 128) return launch<128>(a, stream);
   if (g.head_dim == 64) return launch<64>(a, stream);
   return cudaErrorInvalidValue;

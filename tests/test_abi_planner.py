@@ -241,11 +241,24 @@ def test_append_host_validation():
     lib = pkv.load_library()
     one = ctypes.c_int32(0)
     p = ctypes.cast(ctypes.pointer(one), ctypes.c_void_p)  # a host address: never dereferenced on these paths
-    args = lambda nnz, hk, d, dv, ps, pages, ptr: (ptr, ptr, ptr, nnz, ptr, ptr, ptr, 1, hk, d, dv, ps, pages,
-                                                  ptr, ptr, None, None)
+    args = lambda nnz, hk, d, dv, ps, pages, ptr, lay=0: (ptr, ptr, ptr, nnz, ptr, ptr, ptr, 1, hk, d, dv, ps, pages,
+                                                          lay, ptr, ptr, None, None)
     assert lib.pkv_append_kv(*args(0, 1, 64, 64, 16, 4, p)) == pkv.PKV_OK            # nothing to append
     assert lib.pkv_append_kv(*args(-1, 1, 64, 64, 16, 4, p)) == pkv.PKV_EINVAL
     assert lib.pkv_append_kv(*args(4, 1, 12, 64, 16, 4, p)) == pkv.PKV_EUNSUPPORTED  # head_dim not a multiple of 8
     assert lib.pkv_append_kv(*args(4, 1, 64, 64, 0, 4, p)) == pkv.PKV_EINVAL         # page_size 0
+    assert lib.pkv_append_kv(*args(4, 1, 64, 64, 16, 4, p, 2)) == pkv.PKV_EINVAL     # unknown layout
     assert lib.pkv_append_kv(*args(4, 1, 64, 64, 16, 4, None)) == pkv.PKV_EINVAL     # NULL pointers
     assert b"NULL" in lib.pkv_last_error()
+
+
+def test_kv_layout_option():
+    """kv_layout 0 (NHD) and 1 (HND) plan the same schedule; other values are rejected."""
+    p = W.gqa_prefill()
+    a = _plan(p)
+    b = pkv.plan(p.qo_indptr, p.kv_indptr, None, p.kv_last_page_len, p.num_qo_heads, p.num_kv_heads, p.head_dim,
+                 p.page_size, p.causal, p.sm_scale, upload=False, num_sms=148, kv_layout=1)
+    assert np.array_equal(a.work_units(), b.work_units())
+    with pytest.raises(pkv.PkvError):
+        pkv.plan(p.qo_indptr, p.kv_indptr, None, p.kv_last_page_len, p.num_qo_heads, p.num_kv_heads, p.head_dim,
+                 p.page_size, p.causal, p.sm_scale, upload=False, num_sms=148, kv_layout=2)

@@ -439,3 +439,60 @@ def test_cascade_shared_prefix():
     o, l = pkv.cascade_run(pre_plan, suf_plan, q.cuda(), k.cuda(), v.cuda())
     torch.cuda.synchronize()
     assert_parity(o, l, o_ref, l_ref, what="cascade")
+
+
+# --------------------------------------------------------------------------- HND page layout
+
+HND = [
+    # qo_lens, kv_lens, hq, hk, d, page, causal
+    ([70, 200], [70, 200], 8, 2, 128, 16, True),    # page TMA path, boxes of one kv head's 16 slots
+    ([130, 33], [130, 33], 4, 4, 64, 64, True),
+    ([90, 257], [90, 257], 8, 2, 128, 1, True),     # row gather (vector sparsity)
+    ([40, 100], [140, 100], 4, 2, 128, 4, True),    # chunked prefill, row gather
+    ([1, 1, 1], [70, 300, 5], 8, 2, 128, 16, False),  # decode kernel
+]
+
+
+@pytest.mark.parametrize("case", HND, ids=lambda c: f"h{c[2]}_{c[3]}_d{c[4]}_p{c[5]}_q{max(c[0])}")
+def test_hnd_layout(case):
+    """Pools laid out [page, kv head, slot, D] (HND) give the oracle's result on
+    the same pools in NHD order, and bit for bit the NHD run's result."""
+    qo, kv, hq, hk, d, ps, causal = case
+    p = W.make_problem("hnd", qo, kv, num_qo_heads=hq, num_kv_heads=hk, head_dim=d, page_size=ps, causal=causal,
+                       seed=zlib.crc32(str(case).encode()) % 10000)
+    o_n, l_n, _ = gpu_run(p)
+    d_ = to_dev(p)
+    pl = pkv.plan(p.qo_indptr, p.kv_indptr, d_["kv_indices"], p.kv_last_page_len, hq, hk, d, ps, causal, p.sm_scale,
+                  kv_layout=1)
+    k_h = d_["k_cache"].permute(0, 2, 1, 3).contiguous()
+    v_h = d_["v_cache"].permute(0, 2, 1, 3).contiguous()
+    o_h, l_h = pkv.run(pl, d_["q"], k_h, v_h)
+    torch.cuda.synchronize()
+    assert pkv.device_status(pl) == 0
+    assert_parity(o_h, l_h, *oracle_run(p), what=f"hnd {case}")
+    assert torch.equal(o_h, o_n) and torch.equal(l_h, l_n)
+
+
+def test_append_kv_hnd():
+    """Append into HND pools equals the oracle's NHD append, transposed."""
+    ps, hk, d = 16, 4, 128
+    g = np.random.default_rng(11)
+    kv_after, n_new = np.array([40, 3, 17]), np.array([40, 1, 2])
+    n_pages = (kv_after + ps - 1) // ps
+    pool = int(n_pages.sum()) + 2
+    kv_indptr = np.concatenate([[0], np.cumsum(n_pages)]).astype(np.int32)
+    kv_indices = g.permutation(pool)[: int(n_pages.sum())].astype(np.int32)
+    last = (kv_after - (n_pages - 1) * ps).astype(np.int32)
+    append_indptr = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+    nnz = int(n_new.sum())
+    k = torch.from_numpy(g.standard_normal((pool, ps, hk, d))).to(torch.bfloat16)
+    kn = torch.from_numpy(g.standard_normal((nnz, hk, d))).to(torch.bfloat16)
+    k_ref, _ = oracle.append_paged_kv(k, k, kn, kn, append_indptr, kv_indptr, kv_indices, last, ps)
+    kh = k.permute(0, 2, 1, 3).contiguous().cuda()
+    vh = kh.clone()
+    ii = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    pkv.append_kv(kn.cuda(), kn.cuda(), ii(append_indptr), ii(kv_indptr), ii(kv_indices), ii(last), kh, vh,
+                  kv_layout=1)
+    torch.cuda.synchronize()
+    assert torch.equal(kh.cpu(), k_ref.permute(0, 2, 1, 3).contiguous())
+    assert torch.equal(vh.cpu(), k_ref.permute(0, 2, 1, 3).contiguous())
