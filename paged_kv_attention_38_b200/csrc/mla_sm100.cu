@@ -176,7 +176,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
     cp_async_wait<0>();
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
-    if (lane == 0 && n_tiles > 0) {
+    // The whole warp runs the loop (waits, descriptor arithmetic); one elected
+    // lane (always lane 0) issues each tcgen05.mma / commit. Issued from a
+    // single divergent lane, each MMA cost about 100 cycles of issue time, more
+    // than its M = 64 execution time.
+    if (n_tiles > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kRows, kN, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kRows, 256, true);
       const uint64_t dq = sdesc_sw128(smem_u32(sm.q), 16, 1024);
@@ -196,11 +200,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
           const uint32_t d = tmem + (nh ? (16u << 16) : 0u);
 #pragma unroll
           for (int kk = 0; kk < kN / 16; ++kk)
-            umma_bf16(d, dp + ((kk * 32) >> 4), dvv[st] + ((4 * nh * kBlockBytes + kk * 16 * 128) >> 4), idesc_o,
+            umma_bf16_ss_elect(d, dp + ((kk * 32) >> 4), dvv[st] + ((4 * nh * kBlockBytes + kk * 16 * 128) >> 4), idesc_o,
                       (jj > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&sm.o_done);
-        umma_commit(&sm.kv_empty[st]);
+        umma_commit_elect(&sm.o_done);
+        umma_commit_elect(&sm.kv_empty[st]);
       };
       mbar_wait(&sm.q_full, 0, wc);
       for (int j = 0; j < n_tiles; ++j) {
@@ -212,13 +216,13 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
 #pragma unroll
         for (int kk = 0; kk < kDqk / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4;
-          umma_bf16(tmem + kSCol + st * kN, dq + off, dk[st] + off, idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ss_elect(tmem + kSCol + st * kN, dq + off, dk[st] + off, idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&sm.s_full[st]);
+        umma_commit_elect(&sm.s_full[st]);
         if (j >= 1) issue_pv(j - 1);
       }
       issue_pv(n_tiles - 1);
-      umma_commit(&sm.o_final);
+      umma_commit_elect(&sm.o_final);
       mbar_drain(&sm.o_final, 0);
     }
     __syncwarp();
