@@ -216,12 +216,14 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
     std::stable_sort(s.units.begin(), s.units.end(), longest_first);
   }
 
-  // Prefill runs persistent CTAs (one per SM), each over a fixed list of
-  // units. Greedy list scheduling in the longest-first order above: each unit
-  // goes to the CTA with the least work so far, counted in KV tiles plus one
-  // tile for the unit's own start and end. The units are then stored CTA by CTA.
+  // Prefill and MLA prefill run persistent CTAs (one per SM), each over a
+  // fixed list of units. Greedy list scheduling in the longest-first order
+  // above: each unit goes to the CTA with the least work so far, counted in KV
+  // tiles plus one tile for the unit's own start and end. The units are then
+  // stored CTA by CTA.
   int32_t num_ctas = (int32_t)s.units.size();
-  if (s.kind == kKindPrefill && !s.units.empty()) {
+  if ((s.kind == kKindPrefill || s.kind == kKindMla) && !s.units.empty()) {
+    const int32_t tile = s.kind == kKindMla ? 64 : kBlockN;
     num_ctas = (int32_t)std::min<size_t>((size_t)num_sms, s.units.size());
     using Load = std::pair<int64_t, int32_t>;  // (work so far, cta)
     std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
@@ -231,7 +233,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
       Load top = heap.top();
       heap.pop();
       lists[(size_t)top.second].push_back(u);
-      top.first += (u.kv_hi - u.kv_lo + kBlockN - 1) / kBlockN + 1;
+      top.first += (u.kv_hi - u.kv_lo + tile - 1) / tile + 1;
       heap.push(top);
     }
     s.units.clear();

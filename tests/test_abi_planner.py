@@ -164,7 +164,7 @@ def test_longest_units_first():
 
 
 @pytest.mark.parametrize("maker,banded", [(W.gqa_prefill, False), (lambda: W.sparse_vs_dense(16, 2048, True), True),
-                                          (W.tiny_prefill, False)])
+                                          (W.tiny_prefill, False), (W.mla_prefill, False)])
 def test_persistent_prefill_schedule(maker, banded):
     """Prefill: min(SMs, units) persistent CTAs; every unit in exactly one CTA's
     list and the greedy balance bound: the loads (KV tiles + 1 per unit)
@@ -173,12 +173,17 @@ def test_persistent_prefill_schedule(maker, banded):
     134 MB) it is instead ordered band by band, i.e. by (request, kv head)
     group, so that concurrently running units share groups."""
     p = maker()
-    pl = _plan(p)
+    if p.is_mla:
+        pl = pkv.plan_mla(p.qo_indptr, p.kv_indptr, None, p.kv_last_page_len, p.num_qo_heads, 512, 64, p.page_size,
+                          p.causal, p.sm_scale, upload=False, num_sms=148)
+    else:
+        pl = _plan(p)
+    tile = 64 if p.is_mla else 128
     u = pl.work_units()
     ptr = pl.cta_units()
     assert pl.num_ctas == min(148, len(u)) == len(ptr) - 1
     assert ptr[0] == 0 and ptr[-1] == len(u) and np.all(np.diff(ptr) >= 1)
-    cost = (u[:, 5] - u[:, 4] + 127) // 128 + 1
+    cost = (u[:, 5] - u[:, 4] + tile - 1) // tile + 1
     loads = np.array([cost[a:b].sum() for a, b in zip(ptr[:-1], ptr[1:])])
     group = u[:, 0].astype(np.int64) * p.num_kv_heads + u[:, 1]
     # bands: whole groups in (request, kv head) order, cut once a band holds >= 148 units
