@@ -216,6 +216,15 @@ PKV_API pkv_status pkv_decode_noalloc(const void* q, const void* k_cache, const 
                                       int32_t num_kv_heads, int32_t head_dim, int32_t page_size,
                                       int32_t max_kv_len, float sm_scale, void* o, float* lse, void* stream);
 
+/* Self-test of the bounded device-side waits (no GPU fault involved): one CTA
+ * waits on an mbarrier that nothing arrives on, through the same bounded wait
+ * every kernel uses. Expected on return (after about 2 s): *status (DEVICE
+ * int32, zero on entry) = 1, the wait-timeout code; times[0] (DEVICE int64) =
+ * nanoseconds the first wait took before giving up (about 2e9); times[1] = the
+ * nanoseconds a second wait took once the CTA was aborting (a few hundred),
+ * or -1 where a wait unexpectedly completed. The CUDA context stays usable. */
+PKV_API pkv_status pkv_selftest_wait_timeout(int32_t* status, int64_t* times, void* stream);
+
 /* Read the device status word of the plan's workspace (synchronises `stream`).
  * PKV_OK if no kernel reported an error; PKV_EDEVICE otherwise (and the code is
  * stored in *code if code != NULL). */

@@ -69,6 +69,7 @@ _SIGS = {
     "pkv_plan_merge_tasks": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
     "pkv_plan_cta_units": (ctypes.c_int32, [_P, _I32P, ctypes.c_int32]),
     "pkv_merge_state_bf16": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
+    "pkv_selftest_wait_timeout": (ctypes.c_int, [_P, _P, _P]),
     "pkv_append_kv": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P, _P, _P] + [ctypes.c_int32] * 7 + [_P, _P, _P, _P]),
     "pkv_plan_destroy": (None, [_P]),
     "pkv_last_error": (ctypes.c_char_p, []),
