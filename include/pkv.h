@@ -135,7 +135,10 @@ PKV_API pkv_status pkv_plan_upload(pkv_plan* plan, void* workspace, size_t works
 /* Run GQA / MHA attention (prefill or decode, chosen by the plan) on `stream`.
  * q, k_cache, v_cache: DEVICE bf16 as laid out above; num_pages = pool size
  * (page ids in kv_indices must be < num_pages; they are not checked on the
- * device). o: DEVICE bf16, lse: DEVICE fp32 (may be NULL to skip it). */
+ * device). o: DEVICE bf16, lse: DEVICE fp32 (may be NULL to skip it).
+ * Threading: one process per GPU. The kernels' shared-memory limit is raised
+ * once per process, so a second device driven by the same process gets a
+ * launch error (PKV_ECUDA), never a wrong result. */
 PKV_API pkv_status pkv_run(const pkv_plan* plan, const void* q, const void* k_cache, const void* v_cache,
                    int32_t num_pages, void* o, float* lse, void* stream);
 
