@@ -267,3 +267,50 @@ def test_kv_layout_option():
     with pytest.raises(pkv.PkvError):
         pkv.plan(p.qo_indptr, p.kv_indptr, None, p.kv_last_page_len, p.num_qo_heads, p.num_kv_heads, p.head_dim,
                  p.page_size, p.causal, p.sm_scale, upload=False, num_sms=148, kv_layout=2)
+
+
+@pytest.mark.parametrize("trial", range(40))
+def test_planner_random_batches(trial):
+    """Seeded random batches over every plan kind (GQA prefill, decode, MLA
+    prefill, MLA decode), page sizes, causal flags, SM counts and forced KV
+    chunks: the work list covers every packed row exactly once with key ranges
+    that partition what the rows can see, the merge list matches the split
+    units, and persistent plans deal every unit to exactly one CTA within the
+    greedy balance bound."""
+    g = np.random.default_rng(1000 + trial)
+    kind = trial % 4
+    batch = int(g.integers(1, 7))
+    ps = int(2 ** g.integers(0, 7))
+    causal = bool(g.integers(0, 2))
+    sms = int(g.choice([1, 7, 64, 148]))
+    chunk = int(g.choice([0, 0, 64, 200, 777]))
+    kv = g.integers(0, 900, size=batch)
+    if kind in (1, 3):  # one query token per request
+        qo = np.ones(batch, dtype=np.int64)
+        causal = False
+    else:
+        qo = np.minimum(g.integers(0, 300, size=batch), np.maximum(kv, 1)) if causal else g.integers(0, 300, size=batch)
+    if kind >= 2:
+        p = W.make_mla_problem("rnd", qo, kv, num_heads=int(g.choice([4, 8, 16])), page_size=ps, causal=causal,
+                               seed=trial)
+        pl = pkv.plan_mla(p.qo_indptr, p.kv_indptr, None, p.kv_last_page_len, p.num_qo_heads, 512, 64, ps, causal,
+                          p.sm_scale, upload=False, num_sms=sms, kv_chunk=chunk)
+        assert pl.kind == (pkv.KIND_MLA_DECODE if kind == 3 else pkv.KIND_MLA)
+    else:
+        hk = int(g.choice([1, 2, 4]))
+        hq = hk * int(g.choice([1, 2, 4, 8] if kind == 1 else [1, 3, 4, 16]))
+        p = _lengths_problem(qo, kv, hq=hq, hk=hk, ps=ps, causal=causal)
+        pl = _plan(p, num_sms=sms, kv_chunk=chunk)
+        assert pl.kind == (pkv.KIND_DECODE if kind == 1 else pkv.KIND_PREFILL)
+    _check_coverage(p, pl)
+    ptr = pl.cta_units()
+    if pl.kind in (pkv.KIND_PREFILL, pkv.KIND_MLA) and pl.num_units > 0:
+        u = pl.work_units()
+        assert len(ptr) == pl.num_ctas + 1 == min(sms, len(u)) + 1
+        assert ptr[0] == 0 and ptr[-1] == len(u) and np.all(np.diff(ptr) >= 1)
+        tile = 64 if pl.kind == pkv.KIND_MLA else 128
+        cost = (u[:, 5] - u[:, 4] + tile - 1) // tile + 1
+        loads = np.array([cost[a:b].sum() for a, b in zip(ptr[:-1], ptr[1:])])
+        assert loads.max() - loads.min() <= cost.max()
+    else:
+        assert ptr.size == 0 and pl.num_ctas == pl.num_units
