@@ -6,12 +6,15 @@
 //   LSE = log2(sum_i 2^LSE_i),   O = sum_i 2^(LSE_i - LSE) O_i.
 // The split-KV schedule (discussion #15, disable_split_kv) relies on it.
 //
-// One warp per output row: each lane reads every part's LSE (a handful of
-// floats), then strides over the row's columns. A task's rows are spread over
-// blockIdx.y as well, so a few tasks with many rows (MLA decode: 16 heads x 512
-// columns x tens of parts) still fill the GPU. The reads are coalesced along
-// the row; the data is read once, so the kernel is bound by HBM traffic of
-// the partials (tiny next to the KV stream that produced them).
+// One warp per (output row, 128-column segment): each lane reads every
+// part's LSE (a handful of floats, cached), then 4 columns of every part.
+// A task's rows and segments are spread over blockIdx.y as well, so a few
+// tasks with many rows (MLA decode: 16 heads x 512 columns x ~10 parts) still
+// give thousands of warps, and the loops over parts are unrolled so that a
+// warp's loads of several parts are in flight together (one part per
+// iteration waited a full memory latency per part). The reads are coalesced
+// along the row and the data is read once, so the kernel is bound by HBM
+// traffic of the partials (small next to the KV stream that produced them).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -26,6 +29,7 @@ constexpr int kWarps = 4;
 
 __device__ __forceinline__ float part_max(const float* lse, size_t stride, int num) {
   float m = -INFINITY;
+#pragma unroll 8
   for (int i = 0; i < num; ++i) m = fmaxf(m, lse[i * stride]);
   return m;
 }
@@ -42,20 +46,27 @@ __global__ void __launch_bounds__(kWarps * 32) merge_tasks_kernel(const MergeTas
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Dv = g.head_dim_v, G = g.group, R = g.part_rows;
   const size_t slot_stride = (size_t)R;
-  for (int r = blockIdx.y * kWarps + warp; r < t.rows; r += gridDim.y * kWarps) {
+  const int segs = (Dv + 127) / 128;
+  for (int item = blockIdx.y * kWarps + warp; item < t.rows * segs; item += gridDim.y * kWarps) {
+    const int r = item / segs, seg = item - r * segs;
     const float* lp = part_lse + (size_t)t.slot0 * R + r;
     const float m = part_max(lp, slot_stride, t.num);
     const float mu = m == -INFINITY ? 0.f : m;
     float L = 0.f;
+#pragma unroll 8
     for (int i = 0; i < t.num; ++i) L += ex2(lp[i * slot_stride] - mu);
     const float inv = L > 0.f ? 1.f / L : 0.f;
     const int pr = t.row0 + r;
     const size_t orow = (size_t)(req.q_start + pr / G) * g.num_qo_heads + t.kv_head * G + pr % G;
-    for (int d = lane * 4; d < Dv; d += 128) {
+    const int d = seg * 128 + lane * 4;
+    if (d < Dv) {
+      const float* op = part_o + ((size_t)t.slot0 * R + r) * Dv + d;
+      const size_t part_stride = (size_t)R * Dv;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
       for (int i = 0; i < t.num; ++i) {
         const float w = ex2(lp[i * slot_stride] - mu);
-        const float4 x = *reinterpret_cast<const float4*>(part_o + (((size_t)(t.slot0 + i) * R + r) * Dv + d));
+        const float4 x = *reinterpret_cast<const float4*>(op + i * part_stride);
         acc.x += w * x.x;
         acc.y += w * x.y;
         acc.z += w * x.z;
@@ -66,7 +77,7 @@ __global__ void __launch_bounds__(kWarps * 32) merge_tasks_kernel(const MergeTas
       packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
       *reinterpret_cast<uint2*>(o + orow * Dv + d) = packed;
     }
-    if (lane == 0 && lse) lse[orow] = L > 0.f ? mu + __log2f(L) : -INFINITY;
+    if (lane == 0 && seg == 0 && lse) lse[orow] = L > 0.f ? mu + __log2f(L) : -INFINITY;
   }
 }
 
@@ -120,7 +131,8 @@ __global__ void merge_states_kernel(const float* o_parts, const float* lse_parts
 cudaError_t launch_merge_tasks(const LaunchGeom& g, const DeviceView& dv, void* o, float* lse,
                                cudaStream_t stream) {
   if (g.num_merge == 0) return cudaSuccess;
-  const dim3 grid(g.num_merge, (g.part_rows + kWarps - 1) / kWarps);
+  const int segs = (g.head_dim_v + 127) / 128;
+  const dim3 grid(g.num_merge, (g.part_rows * segs + kWarps - 1) / kWarps);
   merge_tasks_kernel<<<grid, kWarps * 32, 0, stream>>>(dv.merges, g, dv.reqs, dv.part_o, dv.part_lse,
                                                        static_cast<__nv_bfloat16*>(o), lse);
   return cudaGetLastError();
