@@ -13,6 +13,8 @@ from .paged_ref import (  # noqa: F401
     LN2,
     append_paged_kv,
     attend,
+    dequantize_kv,
+    e4m3_to_f64,
     gather_pages,
     kv_lengths,
     merge_state,
@@ -21,6 +23,7 @@ from .paged_ref import (  # noqa: F401
     mla_paged_attention,
     mla_paged_attention_rows,
     paged_attention,
+    paged_attention_quantized_kv,
     paged_attention_rows,
     softmax_rows,
     visible,

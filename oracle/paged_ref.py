@@ -35,6 +35,11 @@ What it computes, and where the pages say so
   append optimization"; documentation, ``get_batch_indices_positions``): the
   page table given is the one after the append, so request ``b``'s ``n`` new
   rows take its last ``n`` positions ``kv_len - n .. kv_len - 1``.
+* A per-head-scale quantised KV cache ("[Roadmap] FlashInfer v0.2 to v0.3",
+  milestone "Per Head Scale Quantized KV-Cache"; the documentation lists FP8
+  KV-cache writers such as ``cake_fused_qk_rope_fp8_append``): the pools hold
+  FP8 E4M3 codes and every kv head ``h`` has one fp32 scale for K and one for
+  V; the cache's value is ``decode(code) * scale[h]`` (reading 6).
 
 Readings where the pages are silent (each pinned by a test)
 ------------------------------------------------------------
@@ -46,6 +51,11 @@ Readings where the pages are silent (each pinned by a test)
 4. A query row that sees no key (empty request, or causal with
    ``qo_len > kv_len``) has output 0 and LSE ``-inf``.
 5. Decode is the same function with one query per request and ``causal=False``.
+6. The quantised cache's codes are FP8 E4M3 as the OCP 8-bit floating-point
+   specification defines it (1 sign bit, 4 exponent bits with bias 7, 3
+   mantissa bits; exponent field 0 is subnormal, ``m/8 * 2^-6``; no
+   infinities; ``S.1111.111`` is NaN; largest finite value 448), and attention
+   over it is reading 1 applied to the dequantised K and V.
 """
 from __future__ import annotations
 
@@ -286,3 +296,32 @@ def append_paged_kv(k_cache, v_cache, k_new, v_new, append_indptr, kv_indptr, kv
             k_out[page, slot] = k_new[a0 + i]
             v_out[page, slot] = v_new[a0 + i]
     return k_out, v_out
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """FP8 E4M3 codes (uint8) -> float64 values (reading 6), field by field."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where((c >> 7) & 1, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 0xF) & (c & 0x7 == 0x7), np.nan, mag)
+    return sign * mag
+
+
+def dequantize_kv(codes, scale) -> np.ndarray:
+    """A quantised pool ``[pages, page_size, Hk, D]`` of E4M3 codes with one scale
+    per kv head -> its float64 values, ``decode(code) * scale[h]``."""
+    c = codes.detach().cpu().numpy() if hasattr(codes, "detach") else np.asarray(codes)
+    vals = e4m3_to_f64(c.view(np.uint8) if c.dtype != np.uint8 else c)
+    sc = _f64(scale).reshape(-1)
+    assert sc.shape[0] == vals.shape[2], "one scale per kv head"
+    return vals * sc[None, None, :, None]
+
+
+def paged_attention_quantized_kv(q, k_codes, v_codes, k_scale, v_scale, qo_indptr, kv_indptr, kv_indices,
+                                 kv_last_page_len, page_size: int, causal: bool, sm_scale: float, requests=None):
+    """Paged attention over a per-head-scale FP8 E4M3 KV cache (NHD pools):
+    the dequantised pools through ``paged_attention``."""
+    return paged_attention(q, dequantize_kv(k_codes, k_scale), dequantize_kv(v_codes, v_scale), qo_indptr,
+                           kv_indptr, kv_indices, kv_last_page_len, page_size, causal, sm_scale, requests)

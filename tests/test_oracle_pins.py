@@ -592,3 +592,107 @@ def test_cascade_identity():
                                     scale)
     o, lse = oracle.merge_state(o1, l1, o2, l2)
     assert np.abs(o - o_ref).max() < 1e-12 and np.abs(lse - l_ref).max() < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# per-head-scale FP8 E4M3 KV cache
+# ---------------------------------------------------------------------------
+
+def test_e4m3_decode_against_format_and_library():
+    """Every one of the 256 codes against torch's float8_e4m3fn (a library
+    decoder) and a few values fixed by the format itself."""
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_to_f64(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(lib))
+    assert np.isnan(ours).sum() == 2  # S.1111.111 only
+    ok = ~np.isnan(lib)
+    assert np.array_equal(ours[ok], lib[ok])
+    fixed = {0x00: 0.0, 0x38: 1.0, 0xB8: -1.0, 0x7E: 448.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9,
+             0x08: 2.0 ** -6, 0x3C: 1.5, 0x40: 2.0, 0xC4: -3.0}
+    for c, val in fixed.items():
+        assert ours[c] == val, hex(c)
+
+
+def _fp8_codes(shape, gen):
+    """E4M3 codes of N(0, 1) values (no NaN codes), as uint8."""
+    x = torch.randn(shape, generator=gen, dtype=torch.float32)
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def test_quantized_kv_brute_force_per_head_scales():
+    """Distinct per-head scales: the oracle against plain loops that decode each
+    code with torch and multiply by its own head's scale."""
+    gen = torch.Generator().manual_seed(7)
+    hq, hk, d, p = 4, 2, 8, 4
+    qo, kv = [1, 1, 1], [9, 4, 13]
+    pb = _small(11, qo, kv, hq, hk, d, p, False)
+    kc = _fp8_codes(tuple(pb.k_cache.shape), gen)
+    vc = _fp8_codes(tuple(pb.v_cache.shape), gen)
+    ks = torch.tensor([0.5, 3.0], dtype=torch.float32)
+    vs = torch.tensor([2.0, 0.25], dtype=torch.float32)
+    kd = kc.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    vd = vc.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    k_ref, v_ref = np.zeros(kd.shape), np.zeros(vd.shape)
+    for pg in range(kd.shape[0]):
+        for s in range(p):
+            for h in range(hk):
+                for x in range(d):
+                    k_ref[pg, s, h, x] = kd[pg, s, h, x] * float(ks[h])
+                    v_ref[pg, s, h, x] = vd[pg, s, h, x] * float(vs[h])
+    o_bf, l_bf = brute_force(_f64(pb.q), k_ref, v_ref, pb.qo_indptr, pb.kv_indptr, pb.kv_indices,
+                             pb.kv_last_page_len, p, False, pb.sm_scale)
+    o, lse = oracle.paged_attention_quantized_kv(pb.q, kc, vc, ks, vs, pb.qo_indptr, pb.kv_indptr, pb.kv_indices,
+                                                 pb.kv_last_page_len, p, False, pb.sm_scale)
+    assert np.abs(o - o_bf).max() < 1e-12 and np.abs(lse - l_bf).max() < 1e-12
+
+
+def test_quantized_kv_scale_laws():
+    """A V scale multiplies O and leaves the LSE; a K scale acts as a factor on
+    sm_scale; unit scales reduce to attention over the decoded codes."""
+    gen = torch.Generator().manual_seed(8)
+    pb = _small(12, [1, 1], [37, 5], 8, 2, 16, 16, False)
+    kc = _fp8_codes(tuple(pb.k_cache.shape), gen)
+    vc = _fp8_codes(tuple(pb.v_cache.shape), gen)
+    one = torch.ones(2)
+    args = (pb.qo_indptr, pb.kv_indptr, pb.kv_indices, pb.kv_last_page_len, 16, False)
+    o1, l1 = oracle.paged_attention_quantized_kv(pb.q, kc, vc, one, one, *args, pb.sm_scale)
+    o2, l2 = oracle.paged_attention_quantized_kv(pb.q, kc, vc, one, torch.tensor([3.0, 3.0]), *args, pb.sm_scale)
+    assert np.abs(o2 - 3.0 * o1).max() < 1e-12 and np.abs(l2 - l1).max() == 0.0
+    o3, l3 = oracle.paged_attention_quantized_kv(pb.q, kc, vc, torch.tensor([0.75, 0.75]), one, *args, pb.sm_scale)
+    o4, l4 = oracle.paged_attention_quantized_kv(pb.q, kc, vc, one, one, *args, pb.sm_scale * 0.75)
+    assert np.abs(o3 - o4).max() < 1e-12 and np.abs(l3 - l4).max() < 1e-12
+    kd = kc.view(torch.float8_e4m3fn).to(torch.float64)
+    vd = vc.view(torch.float8_e4m3fn).to(torch.float64)
+    o5, l5 = oracle.paged_attention(pb.q, kd, vd, *args, pb.sm_scale)
+    assert np.abs(o5 - o1).max() < 1e-12 and np.abs(l5 - l1).max() < 1e-12
+
+
+@pytest.mark.parametrize("kind", ["bias8", "subnormal_as_normal", "scale_by_slot"])
+def test_quantized_pins_catch_planted_mistakes(kind, monkeypatch):
+    """Plausible mistakes planted in a copy of the dequantisation fail a pin."""
+    good_decode, good_dequant = paged_ref.e4m3_to_f64, paged_ref.dequantize_kv
+
+    def decode(codes):
+        c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+        e, m = (c >> 3) & 0xF, (c & 7) / 8.0
+        sign = np.where(c >> 7, -1.0, 1.0)
+        bias = 8.0 if kind == "bias8" else 7.0
+        sub = (1.0 + m) * 2.0 ** (1.0 - bias) if kind == "subnormal_as_normal" else m * 2.0 ** (1.0 - bias)
+        return sign * np.where(e == 0, sub, (1.0 + m) * np.exp2(e - bias))
+
+    def dequant(codes, scale):
+        vals = good_decode(np.asarray(codes))
+        sc = np.asarray(scale, dtype=np.float64)
+        return vals * sc[np.arange(vals.shape[1]) % len(sc)][None, :, None, None]  # by slot, not head
+
+    if kind == "scale_by_slot":
+        monkeypatch.setattr(paged_ref, "dequantize_kv", dequant)
+        test = test_quantized_kv_brute_force_per_head_scales
+    else:
+        monkeypatch.setattr(paged_ref, "e4m3_to_f64", decode)
+        monkeypatch.setattr(oracle, "e4m3_to_f64", decode)
+        test = test_e4m3_decode_against_format_and_library
+    with pytest.raises(AssertionError):
+        test()
+    assert paged_ref.dequantize_kv is (dequant if kind == "scale_by_slot" else good_dequant)
