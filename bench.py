@@ -79,8 +79,9 @@ def decode_bytes(p: W.PagedProblem) -> float:
     if p.is_mla:  # one latent row (ckv | kpe) per key serves as both K and V
         kv = 2 * (p.head_dim + p.head_dim_pe) * int(p.kv_lens.sum())
         q = 2 * p.total_q * p.num_qo_heads * (p.head_dim + p.head_dim_pe)
-    else:
-        kv = 2 * 2 * p.num_kv_heads * p.head_dim * int(p.kv_lens.sum())
+    else:  # K and V, 2 bytes per element (1 for an FP8 cache, plus its scales)
+        el = 1 if p.is_fp8_kv else 2
+        kv = 2 * el * p.num_kv_heads * p.head_dim * int(p.kv_lens.sum()) + (8 * p.num_kv_heads if el == 1 else 0)
         q = 2 * p.total_q * p.num_qo_heads * p.head_dim
     o = 2 * p.total_q * p.num_qo_heads * p.head_dim_v
     lse = 4 * p.total_q * p.num_qo_heads
@@ -228,6 +229,8 @@ class Case:
             self.o = torch.empty(p.total_q, p.num_qo_heads, p.head_dim_v, dtype=torch.bfloat16, device=device)
         else:
             self.q, self.k, self.v = p.q.to(device), p.k_cache.to(device), p.v_cache.to(device)
+            if p.is_fp8_kv:
+                self.k_scale, self.v_scale = p.meta["k_scale"].to(device), p.meta["v_scale"].to(device)
             self.plan = pkv.plan(p.qo_indptr, p.kv_indptr, self.idx, p.kv_last_page_len, p.num_qo_heads,
                                  p.num_kv_heads, p.head_dim, p.page_size, p.causal, p.sm_scale, **plan_kw)
             self.o = torch.empty(p.total_q, p.num_qo_heads, p.head_dim_v, dtype=torch.bfloat16, device=device)
@@ -240,6 +243,8 @@ class Case:
     def run(self):
         if self.p.is_mla:
             pkv.run_mla(self.plan, self.q_nope, self.q_pe, self.ckv, self.kpe, self.o, self.lse)
+        elif self.p.is_fp8_kv:
+            pkv.run_fp8_kv(self.plan, self.q, self.k, self.v, self.k_scale, self.v_scale, self.o, self.lse)
         else:
             pkv.run(self.plan, self.q, self.k, self.v, self.o, self.lse)
 
@@ -460,11 +465,14 @@ def run_ours(args):
     step_ms = pre_ms + dec_ms + (mla_ms or 0.0)
 
     # Rows beyond the step (timed the same way, each alone between L2 flushes):
-    # MLA decode and the paged KV append.
+    # MLA decode, the FP8-KV decode and the paged KV append.
     extra_steps = max(3, min(args.steps, 20))
     mdec = Case(W.mla_decode(shard=rank), device)
     mdec_med, mdec_ms_local = time_case(mdec, flush, extra_steps, 3)
     mdec_ms = max_over_ranks(mdec_ms_local, world)
+    fdec = Case(W.paged_decode_fp8(shard=rank), device)
+    fdec_med, fdec_ms_local = time_case(fdec, flush, extra_steps, 3)
+    fdec_ms = max_over_ranks(fdec_ms_local, world)
     app = AppendCase(W.gqa_prefill(shard=rank), device)
     app_med, app_ms_local = time_case(app, flush, extra_steps, 3)
     app_ms = max_over_ranks(app_ms_local, world)
@@ -502,6 +510,10 @@ def run_ours(args):
         "bound": "hbm", "achieved": round(mdec_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(mdec_gbs / hbm, 4),
         "traffic": profiled_traffic("mla_decode_b64_h16_ckv512_kpe64_ps1.md", MLA_DECODE_SOURCES), "ms": round(mdec_ms, 4),
         "in_step": False}
+    fdec_gbs = decode_bytes(fdec.p) / (fdec_ms * 1e-3) / 1e9
+    roofs["decode_fp8_kernel<128> (b128/h32/kv8/d128/ps16, FP8 E4M3 KV)"] = {
+        "bound": "hbm", "achieved": round(fdec_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(fdec_gbs / hbm, 4),
+        "traffic": None, "ms": round(fdec_ms, 4), "in_step": False}
     app_gbs = app.bytes / (app_ms * 1e-3) / 1e9
     roofs["append_kernel (h16/kv1/d128/ps64 batch)"] = {
         "bound": "hbm", "achieved": round(app_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(app_gbs / hbm, 4),
@@ -559,6 +571,12 @@ def run_ours(args):
                           "bytes": decode_bytes(mdec.p), "units": mdec.plan.num_units, "merges": mdec.plan.num_merges,
                           "workload": "mla_paged_decode_h16_ckv512_kpe64_ps1, batch 64, kv_len U[1024,8192]",
                           "timed": "alone, outside the step, L2 flushed before each launch"}
+    line["decode_fp8"] = {"value": round(fdec_gbs, 1), "unit": "GB/s", "ms": round(fdec_ms, 4),
+                          "bytes": decode_bytes(fdec.p), "units": fdec.plan.num_units,
+                          "merges": fdec.plan.num_merges,
+                          "workload": "paged_decode_b128_h32_kv8_d128_ps16 over an FP8 E4M3 KV cache with "
+                                      "per-kv-head scales, kv_len U[1024,8192]",
+                          "timed": "alone, outside the step, L2 flushed before each launch"}
     line["append"] = {"value": round(app_gbs, 1), "unit": "GB/s", "ms": round(app_ms, 4), "bytes": app.bytes,
                       "rows": app.nnz, "workload": "append of the whole h16/kv1/d128/ps64 prefill batch (K and V)",
                       "timed": "alone, outside the step, L2 flushed before each launch"}
@@ -575,7 +593,7 @@ def run_only(args, device, flush):
               "decode_small": lambda: W.paged_decode(batch=32),
               "sparse": lambda: W.sparse_vs_dense(16, 2048, False),
               "dense": lambda: W.sparse_vs_dense(16, 2048, True),
-              "mla_decode": W.mla_decode}
+              "mla_decode": W.mla_decode, "decode_fp8": W.paged_decode_fp8}
     if args.only == "append":
         c = AppendCase(W.gqa_prefill(), device)
         sampler = ClockSampler(device.index or 0)
@@ -652,7 +670,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--sweep", action="store_true", help="also run the vector-sparse vs dense sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "decode_small", "mla", "mla_decode", "sparse", "dense", "append"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "decode_small", "mla", "mla_decode", "sparse", "dense", "append", "decode_fp8"], default=None,
                     help="time one workload alone (profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -146,6 +146,26 @@ PKV_API pkv_status pkv_run(const pkv_plan* plan, const void* q, const void* k_ca
 PKV_API pkv_status pkv_run_mla(const pkv_plan* plan, const void* q_nope, const void* q_pe, const void* ckv_cache,
                        const void* kpe_cache, int32_t num_pages, void* o, float* lse, void* stream);
 
+/* Paged decode over a per-head-scale quantised KV cache ("[Roadmap]
+ * FlashInfer v0.2 to v0.3", milestone "Per Head Scale Quantized KV-Cache").
+ * The pools hold FP8 E4M3 codes (OCP 8-bit floating point: 1 sign bit, 4
+ * exponent bits with bias 7, 3 mantissa bits, exponent field 0 subnormal,
+ * S.1111.111 NaN), one byte per element, NHD pages:
+ *   k_codes, v_codes  uint8 [num_pages, page_size, num_kv_heads, head_dim]  DEVICE
+ *   k_scale, v_scale  fp32  [num_kv_heads]  DEVICE, or NULL for 1.0
+ * The cache's value is decode(code) * scale[kv head], and the result is
+ * pkv_run's attention over those values: q, o, lse as there. The plan must be
+ * a decode plan from pkv_plan_create (every qo_len <= 1, group <= 16) with the
+ * NHD layout and head_dim 64 or 128; anything else returns PKV_EUNSUPPORTED.
+ * On the device Q is rounded to f16 (|q| must lie within the f16 range) and P
+ * to f16, every code converts exactly to f16, and O and the LSE accumulate in
+ * fp32; NaN codes propagate. Pointers 16-byte aligned; num_pages as in
+ * pkv_run. Never allocates, never synchronises; the split-KV merge runs on the
+ * same stream. */
+PKV_API pkv_status pkv_run_fp8_kv(const pkv_plan* plan, const void* q, const void* k_codes, const void* v_codes,
+                                  const float* k_scale, const float* v_scale, int32_t num_pages, void* o,
+                                  float* lse, void* stream);
+
 /* Merge two attention states over disjoint key sets (all DEVICE fp32):
  * o_a, o_b, o_out [rows, dim]; lse_a, lse_b, lse_out [rows] (base 2).
  * lse_out = log2(2^lse_a + 2^lse_b), o_out = 2^(lse_a-lse_out) o_a + 2^(lse_b-lse_out) o_b.

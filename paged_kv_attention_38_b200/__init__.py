@@ -61,6 +61,7 @@ _SIGS = {
     "pkv_plan_upload": (ctypes.c_int, [_P, _P, ctypes.c_size_t, _P]),
     "pkv_run": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int32, _P, _P, _P]),
     "pkv_run_mla": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int32, _P, _P, _P]),
+    "pkv_run_fp8_kv": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P, _P]),
     "pkv_merge_state": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
     "pkv_merge_states": (ctypes.c_int, [_P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P, _P]),
     "pkv_device_status": (ctypes.c_int, [_P, _P, _I32P]),
@@ -285,6 +286,34 @@ def run_mla(p: Plan, q_nope, q_pe, ckv_cache, kpe_cache, o=None, lse=None, strea
     _check(load_library().pkv_run_mla(p.handle, q_nope.data_ptr(), q_pe.data_ptr(), ckv_cache.data_ptr(),
                                       kpe_cache.data_ptr(), ckv_cache.shape[0], o.data_ptr(), lse.data_ptr(),
                                       _stream_ptr(stream)))
+    return o, lse
+
+
+def run_fp8_kv(p: Plan, q, k_codes, v_codes, k_scale=None, v_scale=None, o=None, lse=None, stream=None):
+    """``pkv_run_fp8_kv``: decode over FP8 E4M3 K/V pools (``torch.float8_e4m3fn``
+    or ``uint8`` codes, NHD) with optional per-kv-head fp32 scales
+    ``[num_kv_heads]``. Returns ``(o bf16 [total_q, Hq, D], lse fp32 [total_q, Hq])``."""
+    import torch
+    _check_tensor(q, "q", torch.bfloat16)
+    for t, n in ((k_codes, "k_codes"), (v_codes, "v_codes")):
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+            raise ValueError(f"{n} must be uint8 or float8_e4m3fn codes")
+        _check_tensor(t, n, t.dtype)
+    hk = k_codes.shape[2]
+    for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        if t is not None:
+            _check_tensor(t, n, torch.float32)
+            if t.numel() != hk:
+                raise ValueError(f"{n} must hold one scale per kv head ({hk})")
+    total_q, hq = q.shape[0], q.shape[1]
+    if o is None:
+        o = torch.empty(total_q, hq, v_codes.shape[-1], dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(total_q, hq, dtype=torch.float32, device=q.device)
+    ptr = lambda t: t.data_ptr() if t is not None else None  # noqa: E731
+    _check(load_library().pkv_run_fp8_kv(p.handle, q.data_ptr(), k_codes.data_ptr(), v_codes.data_ptr(),
+                                         ptr(k_scale), ptr(v_scale), k_codes.shape[0], o.data_ptr(),
+                                         lse.data_ptr(), _stream_ptr(stream)))
     return o, lse
 
 

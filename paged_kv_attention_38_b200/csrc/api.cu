@@ -20,6 +20,8 @@ cudaError_t launch_mla(const LaunchGeom&, const DeviceView&, const int32_t*, con
                        const void*, const void*, void*, float*, cudaStream_t);
 cudaError_t launch_mla_decode(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
                               const void*, const void*, void*, float*, cudaStream_t);
+cudaError_t launch_decode_fp8(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
+                              const void*, const float*, const float*, void*, float*, cudaStream_t);
 cudaError_t launch_merge_tasks(const LaunchGeom&, const DeviceView&, void*, float*, cudaStream_t);
 cudaError_t launch_merge_state(const float*, const float*, const float*, const float*, float*, float*, int, int,
                                cudaStream_t);
@@ -229,6 +231,29 @@ pkv_status pkv_run_mla(const pkv_plan* p, const void* q_nope, const void* q_pe, 
   cudaError_t e = s.kind == kKindMlaDecode
                       ? launch_mla_decode(s.geom, p->dv, p->kv_indices, q_nope, q_pe, ckv_cache, kpe_cache, o, lse, st)
                       : launch_mla(s.geom, p->dv, p->kv_indices, q_nope, q_pe, ckv_cache, kpe_cache, o, lse, st);
+  if (e == cudaSuccess) e = launch_merge_tasks(s.geom, p->dv, o, lse, st);
+  if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return PKV_OK;
+}
+
+pkv_status pkv_run_fp8_kv(const pkv_plan* p, const void* q, const void* k_codes, const void* v_codes,
+                          const float* k_scale, const float* v_scale, int32_t num_pages, void* o, float* lse,
+                          void* stream) {
+  if (!p) return fail(PKV_EINVAL, "plan is NULL");
+  if (!p->uploaded) return fail(PKV_EINVAL, "plan not uploaded (call pkv_plan_upload)");
+  const Schedule& s = p->sched;
+  if (s.kind != kKindDecode)
+    return fail(PKV_EUNSUPPORTED, "FP8 KV cache: decode plans only (every qo_len <= 1, group <= 16)");
+  if (s.geom.kv_layout != 0) return fail(PKV_EUNSUPPORTED, "FP8 KV cache: NHD pages only");
+  if (s.geom.head_dim != 64 && s.geom.head_dim != 128)
+    return fail(PKV_EUNSUPPORTED, "FP8 KV cache: head_dim 64 or 128");
+  if (s.units.empty()) return PKV_OK;
+  if (!q || !k_codes || !v_codes || !o || !p->kv_indices) return fail(PKV_EINVAL, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(o))
+    return fail(PKV_EINVAL, "tensor pointers must be 16-byte aligned");
+  if (num_pages <= 0) return fail(PKV_EINVAL, "num_pages must be positive");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_decode_fp8(s.geom, p->dv, p->kv_indices, q, k_codes, v_codes, k_scale, v_scale, o, lse, st);
   if (e == cudaSuccess) e = launch_merge_tasks(s.geom, p->dv, o, lse, st);
   if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
   return PKV_OK;

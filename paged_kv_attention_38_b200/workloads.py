@@ -100,6 +100,10 @@ class PagedProblem:
     def is_mla(self) -> bool:
         return self.head_dim_pe > 0
 
+    @property
+    def is_fp8_kv(self) -> bool:
+        return self.k_cache is not None and self.k_cache.dtype == torch.uint8
+
 
 def _gen(seed: int) -> torch.Generator:
     g = torch.Generator(device="cpu")
@@ -184,6 +188,39 @@ def make_problem(name: str, qo_lens, kv_lens, *, num_qo_heads: int, num_kv_heads
                         num_qo_heads=num_qo_heads, num_kv_heads=num_kv_heads,
                         head_dim=head_dim, head_dim_v=head_dim_v, causal=causal,
                         sm_scale=sm_scale, q=q, k_cache=k, v_cache=v, seed=seed)
+
+
+def make_fp8_kv_problem(name: str, qo_lens, kv_lens, *, num_qo_heads: int, num_kv_heads: int, head_dim: int,
+                        page_size: int, seed: int, causal: bool = False, sm_scale: Optional[float] = None,
+                        pool_pages: Optional[int] = None) -> PagedProblem:
+    """A GQA paged problem over a per-head-scale FP8 KV cache: ``k_cache`` and
+    ``v_cache`` are uint8 ``[num_pages, P, Hk, D]`` pools of E4M3 codes of N(0, 1)
+    draws, and ``meta`` holds one fp32 scale per kv head for K and for V
+    (``k_scale``, ``v_scale``, uniform in [0.5, 2]). Slots past a request's end
+    hold code 0 in K and the code of 448, the largest E4M3 value, in V."""
+    sm_scale = 1.0 / math.sqrt(head_dim) if sm_scale is None else sm_scale
+    gen = _gen(seed)
+    qo_lens = np.asarray(qo_lens, dtype=np.int64)
+    kv_lens = np.asarray(kv_lens, dtype=np.int64)
+    kv_indptr, kv_indices, last, pool = page_table(kv_lens, page_size, gen, pool_pages)
+    qo_indptr = np.zeros(len(qo_lens) + 1, dtype=np.int32)
+    qo_indptr[1:] = np.cumsum(qo_lens)
+    gen_t = _gen(seed + 100)
+    q = _randn_bf16((int(qo_indptr[-1]), num_qo_heads, head_dim), gen_t)
+    shape = (pool, page_size, num_kv_heads, head_dim)
+    k = torch.randn(*shape, generator=gen_t, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+    v = torch.randn(*shape, generator=gen_t, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)
+    valid = _valid_slot_mask(kv_indptr, kv_indices, last, page_size, pool)
+    k[~valid] = 0
+    v[~valid] = 0x7E
+    k_scale = (0.5 + 1.5 * torch.rand(num_kv_heads, generator=gen_t)).to(torch.float32)
+    v_scale = (0.5 + 1.5 * torch.rand(num_kv_heads, generator=gen_t)).to(torch.float32)
+    return PagedProblem(name=name, qo_indptr=qo_indptr, kv_indptr=kv_indptr,
+                        kv_indices=kv_indices, kv_last_page_len=last, page_size=page_size,
+                        num_qo_heads=num_qo_heads, num_kv_heads=num_kv_heads,
+                        head_dim=head_dim, head_dim_v=head_dim, causal=causal,
+                        sm_scale=sm_scale, q=q, k_cache=k, v_cache=v, seed=seed,
+                        meta={"k_scale": k_scale, "v_scale": v_scale})
 
 
 def make_mla_problem(name: str, qo_lens, kv_lens, *, num_heads: int = 16, head_dim_ckv: int = 512,
@@ -273,6 +310,15 @@ def paged_decode(batch: int = 128, lo: int = 1024, hi: int = 8192, shard: int = 
     return make_problem("paged_decode_b128_h32_kv8_d128_ps16", [1] * batch, kv,
                         num_qo_heads=32, num_kv_heads=8, head_dim=128, page_size=16,
                         causal=False, seed=seed)
+
+
+def paged_decode_fp8(batch: int = 128, lo: int = 1024, hi: int = 8192, shard: int = 0) -> PagedProblem:
+    """The paged decode batch shape (32 qo / 8 kv heads, head_dim 128, page_size
+    16, kv_len ~ U[1024, 8192]) over a per-head-scale FP8 E4M3 KV cache."""
+    seed = SEED_BASE + 8 + 10000 * shard
+    kv = uniform_lengths(batch, lo, hi, _gen(seed + 7))
+    return make_fp8_kv_problem("paged_decode_fp8kv_b128_h32_kv8_d128_ps16", [1] * batch, kv, num_qo_heads=32,
+                               num_kv_heads=8, head_dim=128, page_size=16, seed=seed)
 
 
 def mla_decode(batch: int = 64, lo: int = 1024, hi: int = 8192, shard: int = 0) -> PagedProblem:

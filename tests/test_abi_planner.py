@@ -314,3 +314,28 @@ def test_planner_random_batches(trial):
         assert loads.max() - loads.min() <= cost.max()
     else:
         assert ptr.size == 0 and pl.num_ctas == pl.num_units
+
+
+def test_fp8_kv_workload_and_host_checks():
+    """The FP8-KV decode workload (codes, masked slots, per-head scales), the
+    bench's byte count for it, and the binding's host-side argument checks."""
+    import torch
+    import bench
+    p = W.make_fp8_kv_problem("fp8", [1, 1, 1], [5, 40, 16], num_qo_heads=8, num_kv_heads=2, head_dim=64,
+                              page_size=16, seed=1)
+    assert p.is_fp8_kv and p.k_cache.dtype == torch.uint8 and p.k_cache.shape == (p.num_pages, 16, 2, 64)
+    valid = torch.zeros(p.num_pages, 16, dtype=torch.bool)
+    for b in range(p.batch):
+        for pos in range(int(p.kv_lens[b])):
+            valid[int(p.kv_indices[p.kv_indptr[b] + pos // 16]), pos % 16] = True
+    assert torch.all(p.k_cache[~valid] == 0) and torch.all(p.v_cache[~valid] == 0x7E)
+    codes = p.k_cache[valid]
+    assert not torch.any((codes & 0x7F) == 0x7F), "no NaN codes in valid slots"
+    for s in (p.meta["k_scale"], p.meta["v_scale"]):
+        assert s.shape == (2,) and s.dtype == torch.float32 and torch.all((s >= 0.5) & (s <= 2.0))
+    n_keys = int(p.kv_lens.sum())
+    fixed = 2 * (2 * 3 * 8 * 64) + 4 * 3 * 8 + 4 * len(p.kv_indices)  # Q and O bf16, LSE, page ids
+    assert bench.decode_bytes(p) == 2 * 2 * 64 * n_keys + 8 * 2 + fixed
+    pl_like = object()
+    with pytest.raises(ValueError):
+        pkv.run_fp8_kv(pl_like, p.q, p.k_cache, p.v_cache)  # host tensors are refused before any call

@@ -212,6 +212,86 @@ def test_decode_full_size():
     assert_parity(o, lse, *oracle_run(p), what="decode full")
 
 
+# --------------------------------------------------------------------------- FP8 E4M3 KV decode
+
+def gpu_run_fp8(p: W.PagedProblem, k_scale=True, v_scale=True, **plan_kw):
+    d = to_dev(p)
+    pl = pkv.plan(p.qo_indptr, p.kv_indptr, d["kv_indices"], p.kv_last_page_len, p.num_qo_heads,
+                  p.num_kv_heads, p.head_dim, p.page_size, p.causal, p.sm_scale, **plan_kw)
+    ks = p.meta["k_scale"].cuda() if k_scale else None
+    vs = p.meta["v_scale"].cuda() if v_scale else None
+    o, lse = pkv.run_fp8_kv(pl, d["q"], d["k_cache"], d["v_cache"], ks, vs)
+    torch.cuda.synchronize()
+    assert pkv.device_status(pl) == 0
+    return o, lse, pl
+
+
+def oracle_fp8(p: W.PagedProblem, k_scale=True, v_scale=True):
+    one = torch.ones(p.num_kv_heads)
+    return oracle.paged_attention_quantized_kv(p.q, p.k_cache, p.v_cache, p.meta["k_scale"] if k_scale else one,
+                                               p.meta["v_scale"] if v_scale else one, p.qo_indptr, p.kv_indptr,
+                                               p.kv_indices, p.kv_last_page_len, p.page_size, p.causal, p.sm_scale)
+
+
+FP8_DECODE = [
+    # kv_lens, hq, hk, d, page, forced kv chunk (0 = planner's)
+    ([1, 63, 64, 65, 700, 3000], 32, 8, 128, 16, 0),   # ragged tails, the longest request split
+    ([0, 5, 129, 1000], 8, 8, 64, 1, 64),              # MHA, page_size 1, an empty request, all split
+    ([300, 17], 16, 1, 128, 4, 0),                     # group 16 on one kv head
+]
+
+
+@pytest.mark.parametrize("case", FP8_DECODE, ids=lambda c: f"h{c[1]}_{c[2]}_d{c[3]}_p{c[4]}_k{c[5]}")
+def test_fp8_kv_decode(case):
+    kv, hq, hk, d, ps, chunk = case
+    p = W.make_fp8_kv_problem("fp8dec", [1] * len(kv), kv, num_qo_heads=hq, num_kv_heads=hk, head_dim=d,
+                              page_size=ps, seed=zlib.crc32(str(case).encode()) % 10000)
+    o, lse, pl = gpu_run_fp8(p, **({"kv_chunk": chunk} if chunk else {}))
+    assert pl.kind == pkv.KIND_DECODE
+    if chunk:
+        assert pl.num_merges > 0
+    assert_parity(o, lse, *oracle_fp8(p), what=f"fp8 decode {case}")
+
+
+def test_fp8_kv_decode_unit_scales():
+    """NULL scales read as 1.0."""
+    p = W.make_fp8_kv_problem("fp8dec1", [1, 1], [90, 400], num_qo_heads=8, num_kv_heads=2, head_dim=128,
+                              page_size=16, seed=3)
+    o, lse, _ = gpu_run_fp8(p, k_scale=False, v_scale=False)
+    assert_parity(o, lse, *oracle_fp8(p, k_scale=False, v_scale=False), what="fp8 decode unit scales")
+
+
+def test_fp8_kv_rejects_prefill_plan():
+    p = W.make_fp8_kv_problem("fp8pre", [4, 2], [40, 9], num_qo_heads=4, num_kv_heads=2, head_dim=128,
+                              page_size=16, seed=4)
+    d = to_dev(p)
+    pl = pkv.plan(p.qo_indptr, p.kv_indptr, d["kv_indices"], p.kv_last_page_len, 4, 2, 128, 16, True, p.sm_scale)
+    with pytest.raises(Exception, match="decode plans only"):
+        pkv.run_fp8_kv(pl, d["q"], d["k_cache"], d["v_cache"])
+
+
+@pytest.mark.slow
+def test_fp8_kv_decode_full_size_sampled():
+    """The full FP8 decode batch (b128/h32/kv8/d128/ps16, kv_len U[1024, 8192]) in
+    the bench's launch configuration; 12 requests checked against the oracle on a
+    pool cut down to their own pages."""
+    p = W.paged_decode_fp8()
+    o, lse, pl = gpu_run_fp8(p)
+    assert pl.num_merges > 0
+    rng = np.random.default_rng(9)
+    reqs = sorted({0, p.batch - 1, *rng.integers(0, p.batch, 10).tolist()})
+    pages = [p.kv_indices[p.kv_indptr[b]:p.kv_indptr[b + 1]] for b in reqs]
+    ids = np.concatenate(pages)
+    sub_indptr = np.concatenate([[0], np.cumsum([len(x) for x in pages])]).astype(np.int32)
+    sub_q = torch.stack([p.q[int(p.qo_indptr[b])] for b in reqs])
+    o_ref, l_ref = oracle.paged_attention_quantized_kv(
+        sub_q, p.k_cache[torch.from_numpy(ids.astype(np.int64))], p.v_cache[torch.from_numpy(ids.astype(np.int64))],
+        p.meta["k_scale"], p.meta["v_scale"], np.arange(len(reqs) + 1, dtype=np.int32), sub_indptr,
+        np.arange(len(ids), dtype=np.int32), p.kv_last_page_len[reqs], p.page_size, False, p.sm_scale)
+    rows = [int(p.qo_indptr[b]) for b in reqs]
+    assert_parity(o[rows], lse[rows], o_ref, l_ref, what="fp8 decode full")
+
+
 # --------------------------------------------------------------------------- merge
 
 def test_merge_state_kernels():
