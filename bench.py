@@ -339,28 +339,55 @@ def e2e_prefill(p: W.PagedProblem, device, steps: int, warmup: int):
     return ms, h2d, d2h
 
 
-def cpu_baseline(seconds_target: float = 15.0):
-    """The float64 oracle, as it stands, on a bounded sample of the prefill workload:
-    whole requests of the h16/kv1/d128/ps64 batch, shortest first, until the target
-    CPU time is spent. Returns TFLOP/s on the sample's causal FLOPs."""
+def _blas_threads() -> int:
+    """Threads NumPy's BLAS runs with (the oracle's matmuls), else the CPU affinity."""
+    try:
+        import threadpoolctl
+        n = [p["num_threads"] for p in threadpoolctl.threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except ImportError:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def _oracle_sample(p, order, seconds_target: float):
+    """Whole requests of `p` in `order` through the oracle until the target time is spent."""
     import oracle
-    p = W.gqa_prefill()
-    order = np.argsort(p.qo_lens)
     t0 = time.perf_counter()
     flops, done = 0.0, []
-    for b in order.tolist():
+    for b in order:
         oracle.paged_attention(p.q, p.k_cache, p.v_cache, p.qo_indptr, p.kv_indptr, p.kv_indices,
                                p.kv_last_page_len, p.page_size, True, p.sm_scale, requests=[b])
         L = int(p.qo_lens[b])
         flops += 2.0 * (2 * p.head_dim) * p.num_qo_heads * L * (L + 1) / 2
-        done.append((b, L))
+        done.append(L)
         if time.perf_counter() - t0 > seconds_target:
             break
-    dt = time.perf_counter() - t0
-    cores = len(os.sched_getaffinity(0))
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{len(done)} of 8 requests of the h16/kv1/d128/ps64 prefill batch "
-                      f"(qo_len {[l for _, l in done]}), float64 NumPy, {dt:.1f} s"}
+    return flops, done, time.perf_counter() - t0
+
+
+def cpu_baseline(seconds_target: float = 15.0):
+    """The float64 oracle, as it stands, on a bounded sample of the prefill workload:
+    whole requests of the h16/kv1/d128/ps64 batch, shortest first, until the target
+    CPU time is spent, with every BLAS thread; then the shortest request again with
+    BLAS limited to one thread. Returns TFLOP/s on the sample's causal FLOPs."""
+    p = W.gqa_prefill()
+    order = np.argsort(p.qo_lens).tolist()
+    flops, done, dt = _oracle_sample(p, order, seconds_target)
+    out = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+           "sample": f"{len(done)} of 8 requests of the h16/kv1/d128/ps64 prefill batch "
+                     f"(qo_len {done}), float64 NumPy, {dt:.1f} s",
+           "affinity": len(os.sched_getaffinity(0))}
+    try:
+        import threadpoolctl
+        with threadpoolctl.threadpool_limits(1, user_api="blas"):
+            f1, d1, t1 = _oracle_sample(p, order[:1], 0.0)
+        out["value_1_thread"] = f1 / t1 / 1e12
+        out["sample_1_thread"] = f"the shortest request (qo_len {d1[0]}) with one BLAS thread, {t1:.1f} s"
+    except ImportError:
+        pass
+    return out
 
 
 def dist_setup(n_gpus: int):
@@ -649,7 +676,7 @@ def run_reference(args):
                                p.kv_last_page_len, p.page_size, True, p.sm_scale, requests=[b])
     dt = (time.perf_counter() - t0) / args.steps
     value = flops / dt / 1e12
-    cores = len(os.sched_getaffinity(0))
+    cores = _blas_threads()
     sample = (f"request {b} (qo_len = kv_len = {L}) of the h16/kv1/d128/ps64 prefill batch per step, "
               f"float64 NumPy oracle")
     print(json.dumps({
