@@ -46,7 +46,8 @@
  *   Device pointers must be 16-byte aligned. Slots past kv_last_page_len in a
  *   last page may hold any finite values; they are read but masked.
  *
- * Supported: bf16 only; sm_scale > 0; head_dim 64 or 128 (GQA), 512 + 64 (MLA); page_size a
+ * Supported: bf16 (and FP8 E4M3 K/V pools for decode, pkv_run_fp8_kv);
+ * sm_scale > 0; head_dim 64 or 128 (GQA), 512 + 64 (MLA); page_size a
  * power of two in [1, 256]; num_qo_heads % num_kv_heads == 0 with group size
  * <= 128 (<= 16 on the decode path). Anything else returns PKV_EUNSUPPORTED.
  *
