@@ -240,13 +240,13 @@ pkv_status pkv_run_fp8_kv(const pkv_plan* p, const void* q, const void* k_codes,
                           const float* k_scale, const float* v_scale, int32_t num_pages, void* o, float* lse,
                           void* stream) {
   if (!p) return fail(PKV_EINVAL, "plan is NULL");
-  if (!p->uploaded) return fail(PKV_EINVAL, "plan not uploaded (call pkv_plan_upload)");
   const Schedule& s = p->sched;
   if (s.kind != kKindDecode)
     return fail(PKV_EUNSUPPORTED, "FP8 KV cache: decode plans only (every qo_len <= 1, group <= 16)");
   if (s.geom.kv_layout != 0) return fail(PKV_EUNSUPPORTED, "FP8 KV cache: NHD pages only");
   if (s.geom.head_dim != 64 && s.geom.head_dim != 128)
     return fail(PKV_EUNSUPPORTED, "FP8 KV cache: head_dim 64 or 128");
+  if (!p->uploaded) return fail(PKV_EINVAL, "plan not uploaded (call pkv_plan_upload)");
   if (s.units.empty()) return PKV_OK;
   if (!q || !k_codes || !v_codes || !o || !p->kv_indices) return fail(PKV_EINVAL, "NULL tensor pointer");
   if (!aligned16(q) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(o))

@@ -339,3 +339,25 @@ def test_fp8_kv_workload_and_host_checks():
     pl_like = object()
     with pytest.raises(ValueError):
         pkv.run_fp8_kv(pl_like, p.q, p.k_cache, p.v_cache)  # host tensors are refused before any call
+
+
+def test_fp8_kv_entry_rejects_unsupported_plans():
+    """pkv_run_fp8_kv refuses prefill plans and HND decode plans with
+    PKV_EUNSUPPORTED before touching any pointer, and a decode plan that was
+    never uploaded with PKV_EINVAL."""
+    lib = pkv.load_library()
+    args = [None] * 5 + [1, None, None, None]
+
+    def call(pl):
+        st = lib.pkv_run_fp8_kv(pl.handle, *args)
+        return st, lib.pkv_last_error().decode()
+
+    pre = _plan(W.tiny_prefill())
+    assert pre.kind == pkv.KIND_PREFILL
+    st, msg = call(pre)
+    assert st == 2 and "decode plans only" in msg
+    dec = _lengths_problem([1, 1], [300, 40], hq=8, hk=2, d=128, ps=16, causal=False)
+    st, msg = call(_plan(dec, kv_layout=1))
+    assert st == 2 and "NHD" in msg
+    st, msg = call(_plan(dec))
+    assert st == 1 and "not uploaded" in msg
