@@ -1,6 +1,6 @@
 """Benchmark of the paged-KV attention hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--sweep]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-sweep]
 
 One step = one pass of the hot path over its synthetic batches: the causal
 GQA paged prefill (h16/kv1/d128/ps64, batch 8, lengths U[512, 4096]) and the
@@ -12,6 +12,12 @@ LSE and page indices) rides along under "decode". Kernel times come from CUDA
 events on the launching stream. `e2e` times the same prefill through the
 public API from pinned host buffers: plan + upload, H2D of q / caches / page
 table, run, D2H of O and LSE.
+
+Beside the step (each timed alone between L2 flushes, not in its time): the
+MLA decode, the FP8-KV decode, the paged KV append and, on one GPU, the
+vector-sparse vs dense sweep of the pages' benchmark (`sparse_vs_dense`: page
+size 1 with scattered slots against the contiguous layout of the same problem,
+h32/kv8/d128 causal, every (B, L) of the sweep; `--no-sweep` skips it).
 
 Multi-GPU (torchrun): requests are independent, so every rank runs its own
 batch (weak scaling, no collective on the data path); the timed region is
@@ -92,7 +98,8 @@ def decode_bytes(p: W.PagedProblem) -> float:
 # ----------------------------------------------------------------- profile figures
 
 PREFILL_SOURCES = ("prefill_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
-DECODE_SOURCES = ("decode_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
+DECODE_SOURCES = ("decode_sm100.cu", "decode_core.cuh", "sm100_ptx.cuh", "pkv_internal.h")
+DECODE_FP8_SOURCES = ("decode_fp8_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
 MLA_SOURCES = ("mla_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
 MLA_DECODE_SOURCES = ("mla_decode_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
 APPEND_SOURCES = ("append.cu",)
@@ -540,7 +547,9 @@ def run_ours(args):
     fdec_gbs = decode_bytes(fdec.p) / (fdec_ms * 1e-3) / 1e9
     roofs["decode_fp8_kernel<128> (b128/h32/kv8/d128/ps16, FP8 E4M3 KV)"] = {
         "bound": "hbm", "achieved": round(fdec_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(fdec_gbs / hbm, 4),
-        "traffic": None, "ms": round(fdec_ms, 4), "in_step": False}
+        "traffic": profiled_traffic("decode_fp8_b32_h32_kv8_d128_ps16.md", DECODE_FP8_SOURCES,
+                                    kv_tokens=int(fdec.p.kv_lens.sum())),
+        "ms": round(fdec_ms, 4), "in_step": False}
     app_gbs = app.bytes / (app_ms * 1e-3) / 1e9
     roofs["append_kernel (h16/kv1/d128/ps64 batch)"] = {
         "bound": "hbm", "achieved": round(app_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(app_gbs / hbm, 4),
@@ -609,7 +618,7 @@ def run_ours(args):
                       "timed": "alone, outside the step, L2 flushed before each launch"}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
-    if args.sweep:
+    if world == 1 and not args.no_sweep:
         line["sparse_vs_dense"] = sparse_dense_sweep(device, flush, args)
     print(json.dumps(line), flush=True)
 
@@ -620,7 +629,8 @@ def run_only(args, device, flush):
               "decode_small": lambda: W.paged_decode(batch=32),
               "sparse": lambda: W.sparse_vs_dense(16, 2048, False),
               "dense": lambda: W.sparse_vs_dense(16, 2048, True),
-              "mla_decode": W.mla_decode, "decode_fp8": W.paged_decode_fp8}
+              "mla_decode": W.mla_decode, "decode_fp8": W.paged_decode_fp8,
+              "decode_fp8_small": lambda: W.paged_decode_fp8(batch=32)}
     if args.only == "append":
         c = AppendCase(W.gqa_prefill(), device)
         sampler = ClockSampler(device.index or 0)
@@ -641,19 +651,48 @@ def run_only(args, device, flush):
                       "clocks": sampler.summary()}), flush=True)
 
 
+class DenseCase:
+    """The dense (contiguous ragged) layout of a vector-sparse problem already in
+    HBM: the same queries, and every request's K/V rows gathered on the device into
+    order, described to the kernel as 64-slot pages with the identity page table
+    (every length of the sweep is a multiple of 64)."""
+
+    def __init__(self, sparse: Case):
+        p = sparse.p
+        hk, d = p.num_kv_heads, p.head_dim
+        rows = sparse.idx.long()
+        self.q = sparse.q
+        self.k = sparse.k.view(-1, hk, d)[rows].view(-1, 64, hk, d)
+        self.v = sparse.v.view(-1, hk, d)[rows].view(-1, 64, hk, d)
+        kv_lens = p.kv_lens
+        n_pages = kv_lens // 64
+        kv_indptr = np.concatenate([[0], np.cumsum(n_pages)]).astype(np.int32)
+        self.idx = torch.arange(int(kv_indptr[-1]), dtype=torch.int32, device=self.q.device)
+        self.plan = pkv.plan(p.qo_indptr, kv_indptr, self.idx, np.full(p.batch, 64, np.int32), p.num_qo_heads, hk,
+                             d, 64, True, p.sm_scale)
+        self.o, self.lse = torch.empty_like(sparse.o), torch.empty_like(sparse.lse)
+        self.launches = 1 + (1 if self.plan.num_merges > 0 else 0)
+
+    def run(self):
+        pkv.run(self.plan, self.q, self.k, self.v, self.o, self.lse)
+
+
 def sparse_dense_sweep(device, flush, args):
-    """Vector-sparse (page_size 1, scattered slots) vs contiguous ragged KV, same problem."""
+    """Config 3 of the pages' benchmark: vector-sparse (page_size 1, token slots
+    scattered over the pool) against the dense layout of the same problem, for
+    every (B, L) of the sweep, each timed alone between L2 flushes (median of
+    CUDA-event times). TFLOP/s count the causal FLOPs; ratio = dense time / sparse time."""
     out = []
     for B, L in W.SPARSE_DENSE_SWEEP:
         sp = W.sparse_vs_dense(B, L, contiguous=False)
         cs = Case(sp, device)
-        de = W.sparse_vs_dense(B, L, contiguous=True)
-        cd = Case(de, device)
-        ms_s, _ = time_case(cs, flush, max(5, args.steps), 3)
-        ms_d, _ = time_case(cd, flush, max(5, args.steps), 3)
+        cd = DenseCase(cs)
+        ms_s, _ = time_case(cs, flush, max(10, args.steps), 3)
+        ms_d, _ = time_case(cd, flush, max(10, args.steps), 3)
         f = attention_flops(sp)
         out.append({"B": B, "L": L, "sparse_tflops": round(f / ms_s / 1e9, 1),
-                    "dense_tflops": round(f / ms_d / 1e9, 1), "ratio": round(ms_d / ms_s, 3)})
+                    "dense_tflops": round(f / ms_d / 1e9, 1), "ratio": round(ms_d / ms_s, 3),
+                    "sparse_ms": round(ms_s, 4), "dense_ms": round(ms_d, 4)})
         del cs, cd
         torch.cuda.empty_cache()
     return out
@@ -695,9 +734,12 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--sweep", action="store_true", help="also run the vector-sparse vs dense sweep")
+    ap.add_argument("--sweep", action="store_true",
+                    help="run the vector-sparse vs dense sweep (the default; kept as an alias)")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the vector-sparse vs dense sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "decode_small", "mla", "mla_decode", "sparse", "dense", "append", "decode_fp8"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "decode_small", "mla", "mla_decode", "sparse", "dense", "append",
+                                       "decode_fp8", "decode_fp8_small"], default=None,
                     help="time one workload alone (profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -137,9 +137,8 @@ PKV_API pkv_status pkv_plan_upload(pkv_plan* plan, void* workspace, size_t works
  * q, k_cache, v_cache: DEVICE bf16 as laid out above; num_pages = pool size
  * (page ids in kv_indices must be < num_pages; they are not checked on the
  * device). o: DEVICE bf16, lse: DEVICE fp32 (may be NULL to skip it).
- * Threading: one process per GPU. The kernels' shared-memory limit is raised
- * once per process, so a second device driven by the same process gets a
- * launch error (PKV_ECUDA), never a wrong result. */
+ * Threading: any thread, any device (the kernels' shared-memory limits are
+ * raised once per device, on its first launch). */
 PKV_API pkv_status pkv_run(const pkv_plan* plan, const void* q, const void* k_cache, const void* v_cache,
                    int32_t num_pages, void* o, float* lse, void* stream);
 
@@ -228,9 +227,16 @@ PKV_API pkv_status pkv_append_kv(const void* k_new, const void* v_new, const int
  *   max_kv_len: an upper bound on the requests' kv_len, used to size the split
  *   (a larger kv_len is still computed exactly, only more slowly).
  *   o [batch, num_qo_heads, head_dim] bf16, lse [batch, num_qo_heads] fp32 (or NULL).
- * Supports num_qo_heads / num_kv_heads <= 16, head_dim 64 or 128.
- * Returns PKV_ENOSPACE, without launching anything, when the split would need
- * more than the 16 MiB of scratch. The first call on each device looks up the
+ * Supports num_qo_heads / num_kv_heads <= 16, head_dim 64 or 128, batch and
+ * num_kv_heads up to 65535; q, k_cache, v_cache and o 16-byte aligned, the
+ * index arrays and lse 4-byte aligned (else PKV_EINVAL, nothing launched).
+ * The split gives every SM about four CTAs with chunks of at least 256 keys;
+ * a request whose KV fits one chunk writes O / LSE directly, others go through
+ * the scratch and one merge launch. That rule needs at most about 70 KB of
+ * scratch per SM of the device (about 10 MB on a 148-SM B200), so the
+ * PKV_ENOSPACE refusal (returned without launching anything when a split would
+ * need more than the 16 MiB) can only occur on a GPU with more than 240 SMs.
+ * The first call on each device looks up the
  * scratch address (cudaGetSymbolAddress) and should come before any stream
  * capture. All calls share the scratch: calls whose kernels overlap on the GPU
  * (other streams, unordered threads) race on it and must be serialised. */

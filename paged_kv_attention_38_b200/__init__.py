@@ -26,8 +26,7 @@ __all__ = ["plan", "plan_mla", "run", "run_mla", "merge_state", "merge_states", 
            "Plan", "PkvError", "lib_path", "load_library"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# PKV_LIBRARY may point at another build of the same library (e.g. a tuning variant).
-lib_path = os.environ.get("PKV_LIBRARY") or os.path.join(_HERE, "libpkv.so")
+lib_path = os.path.join(_HERE, "libpkv.so")
 
 PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED, PKV_ENOSPACE, PKV_ECUDA, PKV_EDEVICE = range(6)
 _STATUS = {0: "OK", 1: "EINVAL", 2: "EUNSUPPORTED", 3: "ENOSPACE", 4: "ECUDA", 5: "EDEVICE"}

@@ -1,12 +1,19 @@
 """Build libpkv.so in-tree: nvcc for sm_100a, one shared library, C ABI only.
 
 Usage: python -m paged_kv_attention_38_b200.build  (or build() from Python).
-Objects are compiled in parallel into paged_kv_attention_38_b200/_build/ and
-only recompiled when a source or header is newer than its object.
+Objects are compiled in parallel into paged_kv_attention_38_b200/_build/. An
+object is reused only when a SHA-256 over everything that goes into it (the
+compiler's version, the command line, the source and every header of the
+library) matches the digest stored beside it; the library is relinked unless
+the digest of its objects and link line matches too. File times play no part,
+so a tree copied to another machine with other mtimes rebuilds exactly what
+changed.
 """
 from __future__ import annotations
 
 import concurrent.futures as cf
+import functools
+import hashlib
 import os
 import shutil
 import subprocess
@@ -33,19 +40,49 @@ def _nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
+@functools.lru_cache(maxsize=None)
+def _nvcc_version() -> str:
+    return subprocess.run([_nvcc(), "--version"], capture_output=True, text=True).stdout
+
+
 def _headers():
-    hs = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
+    hs = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh")))
     return hs + [os.path.join(INCLUDE, "pkv.h")]
 
 
-def _compile(src: str, verbose_ptxas: bool) -> str:
+def _digest(cmd, files) -> str:
+    h = hashlib.sha256()
+    h.update(_nvcc_version().encode())
+    h.update("\0".join(cmd).encode())
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def _up_to_date(out: str, digest: str) -> bool:
+    stamp = out + ".sha256"
+    if not (os.path.exists(out) and os.path.exists(stamp)):
+        return False
+    with open(stamp) as f:
+        return f.read().strip() == digest
+
+
+def _stamp(out: str, digest: str) -> None:
+    with open(out + ".sha256", "w") as f:
+        f.write(digest + "\n")
+
+
+def _compile(src: str, verbose_ptxas: bool) -> tuple[str, str]:
     obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-    newest = max([os.path.getmtime(src)] + [os.path.getmtime(h) for h in _headers()])
-    if os.path.exists(obj) and os.path.getmtime(obj) >= newest and not verbose_ptxas:
-        return obj
-    cmd = [_nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
     if src.endswith(".cpp"):
         cmd = [_nvcc(), *FLAGS, "-x", "c++", "-c", src, "-o", obj]
+    else:
+        cmd = [_nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
+    digest = _digest(cmd, [src, *_headers()])
+    if _up_to_date(obj, digest) and not verbose_ptxas:
+        return obj, digest
     if verbose_ptxas and src.endswith(".cu"):
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -53,44 +90,29 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
         raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
     if verbose_ptxas:
         sys.stderr.write(r.stderr)
-    return obj
-
-
-def build_variant(out_lib: str, defines) -> str:
-    """Build a separate copy of the library with extra -D defines (tuning sweeps)."""
-    bdir = os.path.join(os.path.dirname(os.path.abspath(out_lib)), "_build_" + os.path.basename(out_lib))
-    os.makedirs(bdir, exist_ok=True)
-    objs = []
-    for s in SOURCES:
-        src = os.path.join(CSRC, s)
-        obj = os.path.join(bdir, s + ".o")
-        if s.endswith(".cpp"):
-            cmd = [_nvcc(), *FLAGS, "-x", "c++", "-c", src, "-o", obj]
-        else:
-            cmd = [_nvcc(), *ARCH, *FLAGS, *[f"-D{d}" for d in defines], "-c", src, "-o", obj]
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        if r.returncode != 0:
-            raise RuntimeError(f"nvcc failed for {src}:\n{r.stderr}")
-        objs.append(obj)
-    r = subprocess.run([_nvcc(), *ARCH, "-shared", "-o", out_lib, *objs, "-cudart", "static"], capture_output=True, text=True)
-    if r.returncode != 0:
-        raise RuntimeError(r.stderr)
-    return out_lib
+    _stamp(obj, digest)
+    return obj, digest
 
 
 def build(verbose_ptxas: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), srcs))
-    if os.path.exists(LIB) and os.path.getmtime(LIB) >= max(os.path.getmtime(o) for o in objs):
-        return LIB
+        built = list(ex.map(lambda s: _compile(s, verbose_ptxas), srcs))
+    objs = [o for o, _ in built]
     tmp = LIB + ".tmp"
     cmd = [_nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-cudart", "static", "-Xcompiler", "-fPIC"]
+    h = hashlib.sha256("\0".join(cmd).encode())
+    for _, d in built:
+        h.update(d.encode())
+    digest = h.hexdigest()
+    if _up_to_date(LIB, digest):
+        return LIB
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    _stamp(LIB, digest)
     return LIB
 
 

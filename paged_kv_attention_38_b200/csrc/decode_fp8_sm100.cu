@@ -23,6 +23,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "launch_util.h"
 #include "pkv_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -317,10 +318,9 @@ cudaError_t launch(const Args& a, cudaStream_t stream) {
   const size_t comb = (size_t)4 * 16 * D * 4 + 2 * 4 * 16 * 4;
   const size_t smem = pipe > comb ? pipe : comb;
   auto kern = decode_fp8_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   // all of the unified L1 / shared array as shared memory, so three CTAs fit per SM
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = set_smem_attrs_once((const void*)kern, (int)smem, configured, true);
   if (e != cudaSuccess) return e;
   kern<<<a.g.num_units, kThreads, smem, stream>>>(a);
   return cudaGetLastError();

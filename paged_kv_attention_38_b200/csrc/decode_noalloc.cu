@@ -23,10 +23,10 @@
 // clearing, but two calls whose kernels overlap on the GPU (different streams,
 // or one stream shared by several host threads without ordering) race on it.
 //
-// The kernels are a copy of the split-KV decode of decode_sm100.cu in which a
-// CTA takes its (request, kv head, KV chunk) from blockIdx and reads the
-// request's length from the device page table, instead of from an uploaded work
-// list.
+// The attention itself is the planned decode's body (decode::attend in
+// decode_core.cuh); only the CTA's job differs: it takes its (request, kv
+// head, KV chunk) from blockIdx and reads the request's length from the device
+// page table, instead of from an uploaded work list.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -34,6 +34,8 @@
 #include <atomic>
 #include <string>
 
+#include "decode_core.cuh"
+#include "launch_util.h"
 #include "pkv.h"
 #include "pkv_internal.h"
 #include "sm100_ptx.cuh"
@@ -48,9 +50,6 @@ void set_last_error(const std::string& msg);  // api.cu
 
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kStages = 3;
-constexpr int kTile = 64;          // keys per pipeline stage
 constexpr int kRowsMax = 16;       // query heads per kv head handled by one CTA
 constexpr int kMaxDevices = 64;
 
@@ -71,217 +70,49 @@ struct NaArgs {
   float scale;       // sm_scale * log2(e)
 };
 
-template <int D>
-__device__ __forceinline__ uint32_t kv_off(int r, int ch) {
-  return (uint32_t)(r * (D * 2) + ((ch ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ int kv_len_of(const NaArgs& a, int b) {
   const int np = a.kv_indptr[b + 1] - a.kv_indptr[b];
   return np > 0 ? (np - 1) * a.P + a.last_page_len[b] : 0;
 }
 
-// One CTA: request blockIdx.z, kv head blockIdx.y, keys [chunk * blockIdx.x, ...).
+// One CTA: request blockIdx.z, kv head blockIdx.y, keys [chunk * blockIdx.x, ...),
+// through the same attention body as the planned decode kernel.
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2) noalloc_decode_kernel(const __grid_constant__ NaArgs a) {
+__global__ void __launch_bounds__(decode::kThreads, 2) noalloc_decode_kernel(const __grid_constant__ NaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int kTileBytes = kTile * D * 2;
-  constexpr int kChunks = D / 8;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.z, g = blockIdx.y, c = blockIdx.x;
   const int kv_len = kv_len_of(a, b);
   const int kv_lo = c * a.chunk;
   if (c > 0 && kv_lo >= kv_len) return;  // this chunk holds no key; the merge does not read it
   // the last chunk takes every remaining key, so a kv_len above max_kv_len is still exact
   const int kv_hi = c == a.n_chunks - 1 ? kv_len : min(kv_len, kv_lo + a.chunk);
-  const int page0 = a.kv_indptr[b];
-  const int G = a.G, Hk = a.Hk, P = a.P, shift = a.shift;
-  const int n = kv_hi > kv_lo ? (kv_hi - kv_lo + kTile - 1) / kTile : 0;
-  const uint32_t sbase = smem_u32(smem);
-
-  auto load_tile = [&](int j, int stage) {
-    const uint32_t kdst = sbase + stage * 2 * kTileBytes;
-    const uint32_t vdst = kdst + kTileBytes;
-    for (int x = tid; x < kTile * kChunks; x += kThreads) {
-      const int r = x / kChunks, ch = x % kChunks;
-      const int pos = kv_lo + j * kTile + r;
-      const bool ok = pos < kv_hi;
-      size_t off = 0;
-      if (ok) {
-        const int page = __ldg(a.kv_indices + page0 + (pos >> shift));
-        off = (((size_t)page * P + (pos & (P - 1))) * Hk + g) * D + ch * 8;
-      }
-      cp_async_16(kdst + kv_off<D>(r, ch), a.k + off, ok ? 16u : 0u);
-      cp_async_16(vdst + kv_off<D>(r, ch), a.v + off, ok ? 16u : 0u);
-    }
-  };
-#pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
-    if (s < n) load_tile(s, s);
-    cp_async_commit();
+  const size_t row0 = (size_t)b * a.Hq + (size_t)g * a.G;  // first of the group's query / output rows
+  decode::Job jb;
+  jb.q = a.q + row0 * D;
+  jb.k = a.k;
+  jb.v = a.v;
+  jb.pages = a.kv_indices + a.kv_indptr[b];
+  jb.kv_lo = kv_lo;
+  jb.kv_hi = kv_hi;
+  jb.kv_head = g;
+  jb.G = a.G;
+  jb.Hk = a.Hk;
+  jb.P = a.P;
+  jb.shift = a.shift;
+  jb.scale = a.scale;
+  if (a.n_chunks > 1) {
+    const size_t prow = (((size_t)b * a.Hk + g) * a.n_chunks + c) * a.G;
+    jb.part_o = a.part_o + prow * D;
+    jb.part_lse = a.part_lse + prow;
+    jb.o = nullptr;
+    jb.lse = nullptr;
+  } else {
+    jb.part_o = nullptr;
+    jb.part_lse = nullptr;
+    jb.o = a.o + row0 * D;
+    jb.lse = a.lse ? a.lse + row0 : nullptr;
   }
-  uint32_t qa[D / 16][4];
-  {
-    const int r0 = lane >> 2, kq = (lane & 3) * 2;
-    const __nv_bfloat16* qrow = a.q + ((size_t)b * a.Hq + g * G) * D;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      auto ld = [&](int row, int col) -> uint32_t {
-        if (row >= G) return 0u;
-        return *reinterpret_cast<const uint32_t*>(qrow + (size_t)row * D + col);
-      };
-      qa[kk][0] = ld(r0, kk * 16 + kq);
-      qa[kk][1] = ld(r0 + 8, kk * 16 + kq);
-      qa[kk][2] = ld(r0, kk * 16 + kq + 8);
-      qa[kk][3] = ld(r0 + 8, kk * 16 + kq + 8);
-    }
-  }
-  float o_acc[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  for (int j = 0; j < n; ++j) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    if (j + kStages - 1 < n) load_tile(j + kStages - 1, (j + kStages - 1) % kStages);
-    cp_async_commit();
-    const uint32_t kst = sbase + (j % kStages) * 2 * kTileBytes;
-    const uint32_t vst = kst + kTileBytes;
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    {
-      const int mi = lane >> 3;
-      const int row = warp * 16 + (lane & 7) + (mi >> 1) * 8;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kst + kv_off<D>(row, kk * 2 + (mi & 1)), b0, b1, b2, b3);
-        mma16816(s[0], qa[kk], b0, b1);
-        mma16816(s[1], qa[kk], b2, b3);
-      }
-    }
-    const int key0 = kv_lo + j * kTile + warp * 16 + (lane & 3) * 2;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        s[nt][e] = (key0 + nt * 8 + (e & 1)) < kv_hi ? s[nt][e] * a.scale : -INFINITY;
-    float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-    float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-    const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
-    const float a0 = m0 == n0 ? 1.f : ex2(m0 - u0), a1 = m1 == n1 ? 1.f : ex2(m1 - u1);
-    m0 = n0;
-    m1 = n1;
-    float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      s[nt][0] = ex2(s[nt][0] - u0);
-      s[nt][1] = ex2(s[nt][1] - u0);
-      s[nt][2] = ex2(s[nt][2] - u1);
-      s[nt][3] = ex2(s[nt][3] - u1);
-      rs0 += s[nt][0] + s[nt][1];
-      rs1 += s[nt][2] + s[nt][3];
-    }
-    l0 = l0 * a0 + rs0;
-    l1 = l1 * a1 + rs1;
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      o_acc[i][0] *= a0;
-      o_acc[i][1] *= a0;
-      o_acc[i][2] *= a1;
-      o_acc[i][3] *= a1;
-    }
-    uint32_t pa[4];
-    pa[0] = pack_bf16x2(s[0][0], s[0][1]);
-    pa[1] = pack_bf16x2(s[0][2], s[0][3]);
-    pa[2] = pack_bf16x2(s[1][0], s[1][1]);
-    pa[3] = pack_bf16x2(s[1][2], s[1][3]);
-    {
-      const int mi = lane >> 3;
-      const int row = warp * 16 + (lane & 7) + (mi & 1) * 8;
-#pragma unroll
-      for (int np = 0; np < D / 16; ++np) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vst + kv_off<D>(row, np * 2 + (mi >> 1)), b0, b1, b2, b3);
-        mma16816(o_acc[np * 2], pa, b0, b1);
-        mma16816(o_acc[np * 2 + 1], pa, b2, b3);
-      }
-    }
-  }
-  cp_async_wait<0>();
-  __syncthreads();
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  float* so = reinterpret_cast<float*>(smem);
-  float* sm_m = so + 4 * 16 * D;
-  float* sm_l = sm_m + 4 * 16;
-  {
-    const int r0 = lane >> 2, c0 = (lane & 3) * 2;
-    float* ow = so + warp * 16 * D;
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      ow[r0 * D + i * 8 + c0] = o_acc[i][0];
-      ow[r0 * D + i * 8 + c0 + 1] = o_acc[i][1];
-      ow[(r0 + 8) * D + i * 8 + c0] = o_acc[i][2];
-      ow[(r0 + 8) * D + i * 8 + c0 + 1] = o_acc[i][3];
-    }
-    if ((lane & 3) == 0) {
-      sm_m[warp * 16 + r0] = m0;
-      sm_m[warp * 16 + r0 + 8] = m1;
-      sm_l[warp * 16 + r0] = l0;
-      sm_l[warp * 16 + r0 + 8] = l1;
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < G * D; e += kThreads) {
-    const int row = e / D, d = e % D;
-    float mm = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) mm = fmaxf(mm, sm_m[w * 16 + row]);
-    const float mu = mm == -INFINITY ? 0.f : mm;
-    float L = 0.f, acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float wt = ex2(sm_m[w * 16 + row] - mu);
-      L += wt * sm_l[w * 16 + row];
-      acc += wt * so[(w * 16 + row) * D + d];
-    }
-    const float out = L > 0.f ? acc / L : 0.f;
-    const float lse2 = L > 0.f ? mu + __log2f(L) : -INFINITY;
-    if (a.n_chunks > 1) {
-      const size_t prow = (((size_t)b * Hk + g) * a.n_chunks + c) * G + row;
-      a.part_o[prow * D + d] = out;
-      if (d == 0) a.part_lse[prow] = lse2;
-    } else {
-      const size_t orow = (size_t)b * a.Hq + g * G + row;
-      a.o[orow * D + d] = __float2bfloat16_rn(out);
-      if (d == 0 && a.lse) a.lse[orow] = lse2;
-    }
-  }
+  decode::attend<D, false>(smem, jb);
 }
 
 // One CTA per (request, kv head): merge the chunks that hold keys.
@@ -314,21 +145,13 @@ __global__ void __launch_bounds__(128) noalloc_merge_kernel(const __grid_constan
 
 template <int D>
 cudaError_t launch(const NaArgs& a, int batch, cudaStream_t st) {
-  const size_t pipe = (size_t)kStages * 2 * kTile * D * 2;
-  const size_t comb = (size_t)4 * 16 * D * 4 + 2 * 4 * 16 * 4;
-  const size_t smem = pipe > comb ? pipe : comb;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(noalloc_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    // all of the unified L1 / shared array as shared memory, so two CTAs fit per SM
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(noalloc_decode_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                               cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  noalloc_decode_kernel<D><<<dim3(a.n_chunks, a.Hk, batch), kThreads, smem, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  constexpr size_t smem = decode::smem_bytes<D>();
+  // all of the unified L1 / shared array as shared memory, so two CTAs fit per SM
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = set_smem_attrs_once((const void*)noalloc_decode_kernel<D>, (int)smem, configured, true);
+  if (e != cudaSuccess) return e;
+  noalloc_decode_kernel<D><<<dim3(a.n_chunks, a.Hk, batch), decode::kThreads, smem, st>>>(a);
+  e = cudaGetLastError();
   if (e != cudaSuccess || a.n_chunks <= 1) return e;
   noalloc_merge_kernel<D><<<dim3(a.Hk, batch), 128, 0, st>>>(a);
   return cudaGetLastError();
@@ -354,6 +177,16 @@ extern "C" pkv_status pkv_decode_noalloc(const void* q, const void* k_cache, con
     set_last_error("pkv_decode_noalloc: NULL pointer");
     return PKV_EINVAL;
   }
+  // The kernels read q, K and V with 16-byte copies and 4-byte loads and write
+  // O in 2-byte and LSE in 4-byte stores: refuse misaligned pointers on the
+  // host rather than fault on the device.
+  auto aligned = [](const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0; };
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+      !aligned(kv_indptr, 4) || !aligned(kv_indices, 4) || !aligned(kv_last_page_len, 4) ||
+      (lse && !aligned(lse, 4))) {
+    set_last_error("pkv_decode_noalloc: q, k_cache, v_cache and o must be 16-byte aligned, index arrays and lse 4-byte");
+    return PKV_EINVAL;
+  }
   if (num_qo_heads <= 0 || num_kv_heads <= 0 || num_qo_heads % num_kv_heads != 0) {
     set_last_error("pkv_decode_noalloc: num_qo_heads must be a positive multiple of num_kv_heads");
     return PKV_EINVAL;
@@ -361,6 +194,11 @@ extern "C" pkv_status pkv_decode_noalloc(const void* q, const void* k_cache, con
   const int G = num_qo_heads / num_kv_heads;
   if (G > kRowsMax || (head_dim != 64 && head_dim != 128)) {
     set_last_error("pkv_decode_noalloc: needs num_qo_heads / num_kv_heads <= 16 and head_dim 64 or 128");
+    return PKV_EUNSUPPORTED;
+  }
+  // batch and kv heads are grid dimensions y and z of the launches (at most 65535 each)
+  if (batch > 65535 || num_kv_heads > 65535) {
+    set_last_error("pkv_decode_noalloc: batch and num_kv_heads must be at most 65535 per call");
     return PKV_EUNSUPPORTED;
   }
   if (page_size <= 0 || page_size > 256 || (page_size & (page_size - 1)) != 0) {

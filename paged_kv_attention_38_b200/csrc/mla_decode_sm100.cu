@@ -20,6 +20,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "launch_util.h"
 #include "pkv_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -313,16 +314,10 @@ cudaError_t launch_mla_decode(const LaunchGeom& g, const DeviceView& dv, const i
   Args a{static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_pe),
          static_cast<const __nv_bfloat16*>(ckv), static_cast<const __nv_bfloat16*>(kpe), kv_indices,
          static_cast<__nv_bfloat16*>(o), lse, g, dv};
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    // all of the unified L1 / shared array as shared memory, so two CTAs fit per SM
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                               cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // all of the unified L1 / shared array as shared memory, so two CTAs fit per SM
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = set_smem_attrs_once((const void*)mla_decode_kernel, kSmemBytes, configured, true);
+  if (e != cudaSuccess) return e;
   mla_decode_kernel<<<g.num_units, kThreads, kSmemBytes, stream>>>(a);
   return cudaGetLastError();
 }

@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "launch_util.h"
 #include "pkv_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -401,12 +402,9 @@ cudaError_t launch_mla(const LaunchGeom& g, const DeviceView& dv, const int32_t*
          static_cast<const __nv_bfloat16*>(ckv), static_cast<const __nv_bfloat16*>(kpe), kv_indices,
          static_cast<__nv_bfloat16*>(o), lse, g, dv};
   const size_t smem = sizeof(Smem) + 1024;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = set_smem_attrs_once((const void*)mla_kernel, (int)smem, configured, false);
+  if (e != cudaSuccess) return e;
   mla_kernel<<<g.num_ctas, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }

@@ -38,6 +38,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include "launch_util.h"
 #include "pkv_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -696,13 +697,9 @@ bool make_map(CUtensorMap* m, const void* base, int D, int heads, int64_t rows, 
 template <int D, bool kRows, bool kHnd>
 cudaError_t launch_as(const Args& a, cudaStream_t stream) {
   const size_t smem = sizeof(Smem<D>) + 1024;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e =
-        cudaFuncSetAttribute(prefill_kernel<D, kRows, kHnd>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = set_smem_attrs_once((const void*)prefill_kernel<D, kRows, kHnd>, (int)smem, configured, false);
+  if (e != cudaSuccess) return e;
   prefill_kernel<D, kRows, kHnd><<<a.g.num_ctas, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }

@@ -93,6 +93,36 @@ def test_prefill_sweep(case):
     assert_parity(o, lse, *oracle_run(p), what=str(case))
 
 
+# Shapes the header admits beyond the powers of two above. Groups that do not
+# divide the 128-row tile run the cp.async Q loader (packed rows cross token
+# boundaries inside a tile); page sizes 128 and 256 run the TMA path whose box
+# covers a whole KV tile inside one page (page_size >= tile).
+WIDE = [
+    # qo_lens, kv_lens, hq, hk, d, page, causal, forced kv chunk (0 = planner's)
+    ([300, 77], [300, 77], 24, 8, 128, 16, True, 0),        # group 3, ragged tails
+    ([150, 41, 9], [150, 41, 9], 40, 8, 128, 64, True, 0),  # group 5
+    ([100, 260], [100, 260], 12, 1, 64, 8, True, 0),         # group 12 on one kv head
+    ([70, 333], [170, 333], 24, 8, 128, 16, True, 128),     # group 3, chunked prefill, split KV
+    ([1, 1, 1], [500, 33, 2000], 20, 1, 128, 16, False, 0), # group 20 decode batch: the prefill kernel
+    ([200, 37], [200, 300], 16, 4, 128, 128, True, 0),      # page_size 128: one page per KV tile
+    ([300, 129], [300, 129], 16, 4, 128, 256, True, 0),     # page_size 256: two KV tiles per page
+    ([90, 250], [700, 250], 8, 2, 64, 256, True, 128),      # page_size 256, chunks starting mid-page
+    ([160], [160], 12, 4, 128, 128, False, 0),              # group 3 with page_size 128, non-causal
+]
+
+
+@pytest.mark.parametrize("case", WIDE, ids=lambda c: f"h{c[2]}_{c[3]}_d{c[4]}_p{c[5]}_c{int(c[6])}_k{c[7]}")
+def test_prefill_wide_shapes(case):
+    qo, kv, hq, hk, d, ps, causal, chunk = case
+    p = W.make_problem("wide", qo, kv, num_qo_heads=hq, num_kv_heads=hk, head_dim=d, page_size=ps,
+                       causal=causal, seed=zlib.crc32(str(case).encode()) % 10000)
+    o, lse, pl = gpu_run(p, **({"kv_chunk": chunk} if chunk else {}))
+    assert pl.kind == pkv.KIND_PREFILL
+    if chunk:
+        assert pl.num_merges > 0
+    assert_parity(o, lse, *oracle_run(p), what=str(case))
+
+
 @pytest.mark.parametrize("chunk", [128, 384])
 def test_prefill_split_kv_matches(chunk):
     p = W.make_problem("split", [300, 40], [900, 700], num_qo_heads=8, num_kv_heads=2, head_dim=128,
@@ -187,6 +217,10 @@ DECODE_SWEEP = [
     ([500, 1], 16, 1, 128, 64),
     ([129, 700], 8, 8, 64, 1),
     ([2000, 333, 4], 64, 4, 128, 2),
+    ([1, 300, 1000], 24, 8, 128, 16),       # group 3
+    ([77, 513, 2], 40, 8, 64, 128),         # group 5, page_size 128
+    ([2000, 5], 12, 1, 128, 256),           # group 12, page_size 256
+    ([900, 130], 6, 1, 128, 1),             # group 6, vector sparse
 ]
 
 
@@ -530,6 +564,8 @@ HND = [
     ([90, 257], [90, 257], 8, 2, 128, 1, True),     # row gather (vector sparsity)
     ([40, 100], [140, 100], 4, 2, 128, 4, True),    # chunked prefill, row gather
     ([1, 1, 1], [70, 300, 5], 8, 2, 128, 16, False),  # decode kernel
+    ([70, 300], [70, 300], 8, 2, 128, 128, True),   # page_size 128: one kv head's 128 slots per box
+    ([1, 1], [600, 90], 24, 8, 64, 256, False),     # decode, group 3, page_size 256
 ]
 
 

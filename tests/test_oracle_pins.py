@@ -194,6 +194,18 @@ def test_torch_sdpa(hq, hk, qo, kv, causal):
     np.testing.assert_allclose(lse, lse_ref.numpy(), rtol=0, atol=1e-12)
 
 
+def test_oracle_is_deterministic():
+    """The oracle is a pure function of its inputs: two runs on the same seeded
+    problem, one of them after other NumPy work, give bitwise equal results
+    (a nondeterministic oracle, e.g. through threaded BLAS reductions, would make
+    every comparison against it noisy)."""
+    pb = _small(41, [37, 5, 64], [37, 50, 64], 8, 2, 16, 8, True)
+    o1, l1 = _run_oracle(pb)
+    np.linalg.svd(np.random.default_rng(0).standard_normal((300, 300)))  # other BLAS work in between
+    o2, l2 = _run_oracle(pb)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2, equal_nan=True)
+
+
 # ---------------------------------------------------------------------------
 # closed forms
 # ---------------------------------------------------------------------------
