@@ -2,6 +2,7 @@
 // host-to-device copy of a schedule, and the launches behind pkv_run.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -36,7 +37,8 @@ struct pkv_plan {
   Schedule sched;
   const int32_t* kv_indices = nullptr;  // device, borrowed
   // workspace layout (byte offsets)
-  size_t off_status = 0, off_units = 0, off_merges = 0, off_reqs = 0, off_cta = 0, off_lse = 0, off_o = 0, total = 0;
+  size_t off_status = 0, off_units = 0, off_merges = 0, off_reqs = 0, off_cta = 0, off_row0 = 0, off_lse = 0, off_o = 0,
+         off_packed = 0, total = 0;
   size_t staging_bytes = 0;
   void* staging = nullptr;  // host copy of [status | units | merges | reqs | cta_ptr]
   bool staging_pinned = false;
@@ -77,11 +79,16 @@ void layout_workspace(pkv_plan* p) {
   off = align256(off + s.reqs.size() * sizeof(ReqInfo));
   p->off_cta = off;
   off = align256(off + s.cta_ptr.size() * sizeof(int32_t));
+  p->off_row0 = off;
+  off = align256(off + s.kv_row0.size() * sizeof(int32_t));
   p->staging_bytes = off;
   p->off_lse = off;
   off = align256(off + (size_t)s.num_slots * s.geom.part_rows * sizeof(float));
   p->off_o = off;
   off = align256(off + (size_t)s.num_slots * s.geom.part_rows * s.geom.head_dim_v * sizeof(float));
+  p->off_packed = off;
+  if (s.kind == kKindMla)  // the packed latent copy, ckv | kpe per key (at least one row for the tensor map)
+    off = align256(off + (size_t)std::max(1, s.geom.packed_rows) * (s.geom.head_dim + s.geom.head_dim_pe) * 2);
   p->total = off;
 }
 
@@ -179,6 +186,7 @@ pkv_status pkv_plan_upload(pkv_plan* p, void* workspace, size_t bytes, void* str
     if (!s.merges.empty()) std::memcpy(h + p->off_merges, s.merges.data(), s.merges.size() * sizeof(MergeTask));
     if (!s.reqs.empty()) std::memcpy(h + p->off_reqs, s.reqs.data(), s.reqs.size() * sizeof(ReqInfo));
     if (!s.cta_ptr.empty()) std::memcpy(h + p->off_cta, s.cta_ptr.data(), s.cta_ptr.size() * sizeof(int32_t));
+    if (!s.kv_row0.empty()) std::memcpy(h + p->off_row0, s.kv_row0.data(), s.kv_row0.size() * sizeof(int32_t));
   }
   uint8_t* d = static_cast<uint8_t*>(workspace);
   cudaError_t e = cudaMemcpyAsync(d, p->staging, p->staging_bytes, cudaMemcpyHostToDevice,
@@ -191,6 +199,8 @@ pkv_status pkv_plan_upload(pkv_plan* p, void* workspace, size_t bytes, void* str
   p->dv.part_o = reinterpret_cast<float*>(d + p->off_o);
   p->dv.status = reinterpret_cast<int*>(d + p->off_status);
   p->dv.cta_ptr = reinterpret_cast<const int32_t*>(d + p->off_cta);
+  p->dv.kv_row0 = reinterpret_cast<const int32_t*>(d + p->off_row0);
+  p->dv.packed = d + p->off_packed;
   p->uploaded = true;
   return PKV_OK;
 }

@@ -9,87 +9,144 @@
 // i.e. attention with a 576-wide key [ckv | kpe] and a 512-wide value ckv.
 // Output O (bf16, 512 per head) and the base-2 LSE per (token, head).
 //
-// Shape choices for B200. A 128-row tile's 128 x 512 fp32 output alone would
-// fill all 512 TMEM columns, and a 128 x 576 bf16 query tile (144 KB) leaves no
-// room in shared memory for a double-buffered key tile. So a CTA takes 64
-// packed (token, head) rows and 64-key tiles, and runs M = 64 MMAs:
+// Two launches. mla_pack_kernel first copies every latent row a request's
+// page table lists, ckv | kpe (1152 bytes), into a packed copy in the plan's
+// workspace, request by request in key order. With page_size 1 the rows are
+// scattered over the pool one by one, and a 16-byte-copy gather inside the
+// attention kernel could not keep its tensor core fed; packed, each key tile
+// is one dense [keys x 576] block that TMA moves in nine boxes. Every latent
+// row is read by every query tile of its request, so the one pass over the
+// pool (a few MB) is repaid many times; the packed copy stays in L2.
+//
+// mla_kernel then runs the attention. Shape choices for B200. A 128-row
+// tile's 128 x 512 fp32 output alone would fill all 512 TMEM columns, and a
+// 128 x 576 bf16 query tile (144 KB) leaves no room in shared memory for a key
+// ring. So a CTA takes 64 packed (token, head) rows and runs M = 64 MMAs:
 //   TMEM  O rows x latent[0,256)   lanes 16q + [0,16)  (q = sub-partition), cols [0,256)
 //         O rows x latent[256,512) lanes 16q + [16,32),                     cols [0,256)
-//         S (double buffer)        lanes 16q + [0,16),                      cols [256,320), [320,384)
+//         S (double buffer)        lanes 16q + [0,16),                      cols [256,288), [288,320)
 //   (a 64-row accumulator uses half of each 32-lane sub-partition; the two
 //   latent halves of O sit in the two halves, so a warp rescales both with one
 //   32x32b load/store over columns [0,256) without touching S.)
-//   SMEM  Q 64 x 576 (72 KB), a 2-stage ring of 64 x 576 latent rows (K and V
-//   at once: V is the ckv part of the same rows), P 64 x 64 (8 KB).
-// Both MMAs read their operands from shared memory. The kernel is persistent:
-// one CTA per SM runs a host-planned list of units, its barrier phases running
-// on across units, so the next unit's Q and latent rows stream in while the
-// previous unit finishes. Warps: 0-3 softmax and
-// epilogue (lanes 0-15 own S rows and the low O half, lanes 16-31 the high O
-// half of the same rows), 4 TMEM allocator + MMA issuer, 5-8 cp.async gather
-// of Q and of the latent rows through the page table.
+//   SMEM  Q 64 x 576 (72 KB), a 4-stage TMA ring of 32-key latent tiles
+//   (32 x 576, 36 KB: K and V at once, V being the ckv part of the same rows),
+//   P 64 x 32 (in an 8 KB swizzled block).
+// Both MMAs read their operands from shared memory. The tensor core runs a
+// CTA's MMAs in issue order, S(g + 1) then P(g) V(g), so it stays busy while
+// the softmax of a tile runs, and with four stages three tiles are in flight
+// behind the one being consumed. The kernel is persistent: one CTA per SM
+// runs a host-planned list of units, its barrier phases running on across
+// units. Warps: 0-3 softmax and epilogue (lanes 0-15 own S rows and the low O
+// half, lanes 16-31 the high O half of the same rows), 4 TMEM allocator + MMA
+// issuer, 5 TMA producer (one lane).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "launch_util.h"
 #include "pkv_internal.h"
 #include "sm100_ptx.cuh"
+#include "tma_util.h"
 
 namespace pkv {
 
 namespace {
 
 constexpr int kRows = kMlaUnitRows;  // 64
-constexpr int kN = 64;               // keys per tile
+constexpr int kN = 32;               // keys per latent tile
+constexpr int kStages = 4;
 constexpr int kDc = 512;
 constexpr int kDr = 64;
 constexpr int kDqk = kDc + kDr;      // 576
 constexpr int kBlocks = kDqk / 64;   // 9 column blocks of 64 (128-byte rows)
-constexpr int kBlockBytes = kRows * 128;  // one [64 rows x 64] bf16 block: 8 KB
-constexpr int kThreads = 288;
+constexpr int kQBlockBytes = kRows * 128;  // [64 rows x 64] bf16: 8 KB
+constexpr int kKBlockBytes = kN * 128;     // [32 keys x 64] bf16: 4 KB
+constexpr int kStageBytes = kBlocks * kKBlockBytes;
+constexpr int kThreads = 192;
 constexpr int kMmaWarp = 4;
-constexpr int kProdWarp0 = 5;
-constexpr int kProdThreads = 128;
+constexpr int kProdWarp = 5;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol = 256;
 constexpr float kRescaleThreshold = 8.0f;
-static_assert(kN == kRows, "one block shape for Q, latent rows and P");
-
-// Byte offset of 16-byte chunk `ch` (0..71 across the 576-wide row) of row `r`
-// in a [64 x 576] tile held as 9 column blocks of [64 rows x 128 B], 128-byte swizzle.
-__device__ __forceinline__ uint32_t blk_off(int r, int ch) {
-  return (uint32_t)((ch >> 3) * kBlockBytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
-}
 
 struct __align__(1024) Smem {
   __nv_bfloat16 q[kBlocks * kRows * 64];
-  __nv_bfloat16 kv[2][kBlocks * kN * 64];
-  __nv_bfloat16 p[kRows * kN];
+  __nv_bfloat16 kv[kStages][kBlocks * kN * 64];
+  __nv_bfloat16 p[kRows * 64];  // P [64 rows x 32 keys] in the first 64 (logical) bytes of swizzled 128-byte rows
   uint64_t q_full;
   uint64_t q_empty;  // the unit's last QK^T MMAs are done: Q may be overwritten
-  uint64_t kv_full[2];
-  uint64_t kv_empty[2];
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
   uint64_t s_full[2];
   uint64_t s_free[2];
   uint64_t p_full;
   uint64_t o_done;
   uint64_t o_final;
-  int32_t rowsrc[2][kN];  // pool slot of each latent row of the tile in each stage, -1 = zero fill
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(sizeof(Smem) + 1024 <= 232448, "dynamic shared memory of one CTA (227 KB on sm_100)");
 
 struct Args {
-  const __nv_bfloat16* q_nope;
-  const __nv_bfloat16* q_pe;
-  const __nv_bfloat16* ckv;
-  const __nv_bfloat16* kpe;
-  const int32_t* kv_indices;
+  CUtensorMap tm_q;    // q_nope as [total_q * H rows][512]
+  CUtensorMap tm_qpe;  // q_pe as [total_q * H rows][64]
+  CUtensorMap tm_lat;  // packed latent rows [packed_rows][576]
   __nv_bfloat16* o;
   float* lse;
   LaunchGeom g;
   DeviceView dv;
 };
+
+struct PackArgs {
+  const __nv_bfloat16* ckv;
+  const __nv_bfloat16* kpe;
+  const int32_t* kv_indices;
+  const ReqInfo* reqs;
+  const int32_t* kv_row0;
+  __nv_bfloat16* packed;
+  int32_t batch, page_size, page_shift;
+};
+
+// Copy the latent rows of every request with queries into the packed copy:
+// row kv_row0[b] + pos holds ckv (512) then kpe (64) of key pos of request b.
+// A block covers 32 keys of one request (8 warps x 4 keys); a warp moves a
+// 1152-byte row as 72 16-byte pieces, the loads of its four rows first.
+constexpr int kPackKeys = 32;
+__global__ void __launch_bounds__(256) mla_pack_kernel(const __grid_constant__ PackArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int P = a.page_size, shift = a.page_shift;
+  for (int b = blockIdx.y; b < a.batch; b += gridDim.y) {
+    const ReqInfo req = a.reqs[b];
+    if (req.qo_len == 0) continue;
+    const int pos0 = blockIdx.x * kPackKeys + warp * 4;
+    if (pos0 >= req.kv_len) continue;
+    const int row0 = a.kv_row0[b];
+    uint4 v[4][3];
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int pos = pos0 + i;
+      if (pos < req.kv_len) {
+        const size_t src = (size_t)__ldg(a.kv_indices + req.page0 + (pos >> shift)) * P + (pos & (P - 1));
+        const uint4* c = reinterpret_cast<const uint4*>(a.ckv + src * kDc);
+        v[i][0] = __ldg(c + lane);
+        v[i][1] = __ldg(c + 32 + lane);
+        if (lane < 8) v[i][2] = __ldg(reinterpret_cast<const uint4*>(a.kpe + src * kDr) + lane);
+        n = i + 1;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (i < n) {
+        uint4* d = reinterpret_cast<uint4*>(a.packed + (size_t)(row0 + pos0 + i) * kDqk);
+        d[lane] = v[i][0];
+        d[32 + lane] = v[i][1];
+        if (lane < 8) d[64 + lane] = v[i][2];
+      }
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant__ Args a) {
   extern __shared__ uint8_t smem_raw[];
@@ -105,11 +162,13 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
   auto tiles_of = [](const WorkUnit& u) { return (u.kv_hi - u.kv_lo + kN - 1) / kN; };
 
   if (tid == 0) {
-    mbar_init(&sm.q_full, kProdThreads);
+    mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.kv_full[s], kProdThreads);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.s_free[s], 128);
     }
@@ -129,68 +188,48 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
   const uint32_t tmem = sm.tmem_base;
   WaitCtx wc{&sm.abort_flag, a.dv.status};
 
-  if (warp >= kProdWarp0) {
-    // ================================================================ producer
-    const int pt = tid - kProdWarp0 * 32;
-    constexpr int kChunks = kDqk / 8;  // 72 16-byte chunks per 576-wide row
-    const int P = a.g.page_size, shift = a.g.page_shift;
-    int g = 0;   // latent tiles loaded by this CTA (stage g & 1)
-    int uq = 0;  // units with keys whose Q was loaded
-    for (int ui = u_begin; ui < u_end; ++ui) {
-      const WorkUnit unit = a.dv.units[ui];
-      const int n_tiles = tiles_of(unit);
-      if (n_tiles == 0) continue;
-      const ReqInfo req = a.dv.reqs[unit.req];
-      // Q, once the previous unit's QK^T MMAs have read the old one
-      if (uq > 0) mbar_wait(&sm.q_empty, (uq - 1) & 1, wc);
-      for (int c = pt; c < kRows * kChunks; c += kProdThreads) {
-        const int r = c / kChunks, ch = c % kChunks;
-        const bool ok = r < unit.rows;
-        const __nv_bfloat16* src = a.q_nope;
-        if (ok) {
-          const int pr = unit.row0 + r;
-          const size_t row = (size_t)(req.q_start + pr / H) * H + pr % H;
-          src = ch < kDc / 8 ? a.q_nope + row * kDc + ch * 8 : a.q_pe + row * kDr + (ch - kDc / 8) * 8;
+  if (warp == kProdWarp) {
+    // ================================================================ producer (TMA, one lane)
+    if (lane == 0) {
+      tma_prefetch_desc(&a.tm_q);
+      tma_prefetch_desc(&a.tm_qpe);
+      tma_prefetch_desc(&a.tm_lat);
+      int g = 0;   // latent tiles loaded by this CTA (stage g % kStages)
+      int uq = 0;  // units with keys whose Q was loaded
+      for (int ui = u_begin; ui < u_end; ++ui) {
+        const WorkUnit unit = a.dv.units[ui];
+        const int n_tiles = tiles_of(unit);
+        if (n_tiles == 0) continue;
+        const ReqInfo req = a.dv.reqs[unit.req];
+        // Q, once the previous unit's QK^T MMAs have read the old one. The
+        // unit's packed rows are consecutive rows of q viewed as [total_q * H]:
+        // row (token t, head h) of the request is q_start * H + t * H + h.
+        if (uq > 0) mbar_wait(&sm.q_empty, (uq - 1) & 1, wc);
+        mbar_arrive_expect_tx(&sm.q_full, kBlocks * kQBlockBytes);
+        const int qrow = req.q_start * H + unit.row0;
+#pragma unroll
+        for (int blk = 0; blk < kBlocks - 1; ++blk)
+          tma_load_2d(smem_u32(sm.q) + blk * kQBlockBytes, &a.tm_q, &sm.q_full, blk * 64, qrow);
+        tma_load_2d(smem_u32(sm.q) + (kBlocks - 1) * kQBlockBytes, &a.tm_qpe, &sm.q_full, 0, qrow);
+        ++uq;
+        const int krow0 = a.dv.kv_row0[unit.req] + unit.kv_lo;
+        for (int j = 0; j < n_tiles; ++j, ++g) {
+          const int st = g % kStages;
+          if (g >= kStages) mbar_wait(&sm.kv_empty[st], ((g / kStages) - 1) & 1, wc);
+          mbar_arrive_expect_tx(&sm.kv_full[st], kStageBytes);
+          const uint32_t dst = smem_u32(sm.kv[st]);
+#pragma unroll
+          for (int blk = 0; blk < kBlocks; ++blk)
+            tma_load_2d(dst + blk * kKBlockBytes, &a.tm_lat, &sm.kv_full[st], blk * 64, krow0 + j * kN);
         }
-        cp_async_16(smem_u32(sm.q) + blk_off(r, ch), src, ok ? 16u : 0u);
       }
-      cp_async_arrive_noinc(&sm.q_full);
-      ++uq;
-      // Latent tiles: the page lookups of a tile are done once (one row per
-      // thread) into shared memory; then each thread copies a fixed 16-byte
-      // column of every other row: ckv columns 0..63 (two rows per pass), kpe
-      // columns 64..71 (sixteen rows per pass).
-      for (int j = 0; j < n_tiles; ++j, ++g) {
-        const int st = g & 1;
-        if (g >= 2) mbar_wait(&sm.kv_empty[st], ((g >> 1) - 1) & 1, wc);
-        if (pt < kN) {
-          const int pos = unit.kv_lo + j * kN + pt;
-          sm.rowsrc[st][pt] = pos < unit.kv_hi ? __ldg(a.kv_indices + req.page0 + (pos >> shift)) * P + (pos & (P - 1)) : -1;
-        }
-        named_bar_sync(1, kProdThreads);
-        const uint32_t dst = smem_u32(sm.kv[st]);
-        {
-          const int ch = pt & 63;
-          const uint32_t col = (uint32_t)((ch >> 3) * kBlockBytes + ((ch & 7) << 4));
-          for (int r = pt >> 6; r < kN; r += 2) {
-            const int src = sm.rowsrc[st][r];
-            const __nv_bfloat16* gp = src >= 0 ? a.ckv + (size_t)src * kDc + ch * 8 : a.ckv;
-            cp_async_16(dst + r * 128 + (col ^ ((r & 7) << 4)), gp, src >= 0 ? 16u : 0u);
-          }
-        }
-        {
-          const int ch = pt & 7;
-          const uint32_t col = (uint32_t)(8 * kBlockBytes + (ch << 4));
-          for (int r = pt >> 3; r < kN; r += 16) {
-            const int src = sm.rowsrc[st][r];
-            const __nv_bfloat16* gp = src >= 0 ? a.kpe + (size_t)src * kDr + ch * 8 : a.kpe;
-            cp_async_16(dst + r * 128 + (col ^ ((r & 7) << 4)), gp, src >= 0 ? 16u : 0u);
-          }
-        }
-        cp_async_arrive_noinc(&sm.kv_full[st]);
-      }
+      // No TMA write may still land in this CTA's shared memory at exit: only
+      // the last Q and the last kStages tiles can be in flight (every earlier
+      // one was consumed before its buffer was refilled).
+      if (uq > 0) mbar_drain(&sm.q_full, (uq - 1) & 1);
+      for (int k = g - 1; k >= 0 && k >= g - kStages; --k) mbar_drain(&sm.kv_full[k % kStages], (k / kStages) & 1);
     }
-    cp_async_wait<0>();
+    __syncwarp();
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     // The whole warp runs the loop (waits, descriptor arithmetic); one elected
@@ -199,48 +238,48 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
     // than its M = 64 execution time.
     constexpr uint32_t idesc_s = idesc_bf16_f32(kRows, kN, false);
     constexpr uint32_t idesc_o = idesc_bf16_f32(kRows, 256, true);
+    // Descriptors are built once; another stage, block or K-step only moves the
+    // start address, the low 14-bit field (addr >> 4), so offsets are added in place.
     const uint64_t dq = sdesc_sw128(smem_u32(sm.q), 16, 1024);
     const uint64_t dp = sdesc_sw128(smem_u32(sm.p), 16, 1024);
-    uint64_t dk[2], dvv[2];
-    for (int s = 0; s < 2; ++s) {
-      dk[s] = sdesc_sw128(smem_u32(sm.kv[s]), 16, 1024);
-      dvv[s] = sdesc_sw128(smem_u32(sm.kv[s]), kBlockBytes, 1024);
-    }
+    const uint64_t dk0 = sdesc_sw128(smem_u32(sm.kv[0]), 16, 1024);
+    const uint64_t dv0 = sdesc_sw128(smem_u32(sm.kv[0]), kKBlockBytes, 1024);
+    constexpr uint32_t kStageStep = (uint32_t)(kStageBytes >> 4);
     // O += P V for the CTA's latent tile gg; `first`: the unit's first tile
     auto issue_pv = [&](int gg, bool first) {
-      const int st = gg & 1;
+      const int st = gg % kStages;
       mbar_wait(&sm.p_full, gg & 1, wc);
-      fence_proxy_async_smem();
       tc_fence_after();
 #pragma unroll
       for (int nh = 0; nh < 2; ++nh) {
         const uint32_t d = tmem + (nh ? (16u << 16) : 0u);
 #pragma unroll
         for (int kk = 0; kk < kN / 16; ++kk)
-          umma_bf16_ss_elect(d, dp + ((kk * 32) >> 4), dvv[st] + ((4 * nh * kBlockBytes + kk * 16 * 128) >> 4),
-                             idesc_o, (!first || kk > 0) ? 1u : 0u);
+          umma_bf16_ss_elect(d, dp + ((kk * 32) >> 4),
+                             dv0 + st * kStageStep + ((4 * nh * kKBlockBytes + kk * 16 * 128) >> 4), idesc_o,
+                             (!first || kk > 0) ? 1u : 0u);
       }
       umma_commit_elect(&sm.o_done);
       umma_commit_elect(&sm.kv_empty[st]);
     };
-    int g = 0;   // latent tiles of this CTA: stage g & 1 and the per-tile phases
+    int g = 0;   // latent tiles of this CTA: stage g % kStages, S buffer g & 1 and the per-tile phases
     int uq = 0;  // units with keys: q_full / q_empty / o_final phases
     for (int ui = u_begin; ui < u_end; ++ui) {
       const int n_tiles = tiles_of(a.dv.units[ui]);
       if (n_tiles == 0) continue;
       mbar_wait(&sm.q_full, uq & 1, wc);
       for (int j = 0; j < n_tiles; ++j, ++g) {
-        const int st = g & 1;
-        mbar_wait(&sm.kv_full[st], (g >> 1) & 1, wc);
-        if (g >= 2) mbar_wait(&sm.s_free[st], ((g >> 1) - 1) & 1, wc);
-        fence_proxy_async_smem();  // cp.async rows were written through the generic proxy
+        const int st = g % kStages, sb = g & 1;
+        mbar_wait(&sm.kv_full[st], (g / kStages) & 1, wc);
+        if (g >= 2) mbar_wait(&sm.s_free[sb], ((g >> 1) - 1) & 1, wc);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kDqk / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4;
-          umma_bf16_ss_elect(tmem + kSCol + st * kN, dq + off, dk[st] + off, idesc_s, kk > 0 ? 1u : 0u);
+          const uint32_t oq = ((kk >> 2) * kQBlockBytes + (kk & 3) * 32) >> 4;
+          const uint32_t ok = ((kk >> 2) * kKBlockBytes + (kk & 3) * 32) >> 4;
+          umma_bf16_ss_elect(tmem + kSCol + sb * kN, dq + oq, dk0 + st * kStageStep + ok, idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit_elect(&sm.s_full[st]);
+        umma_commit_elect(&sm.s_full[sb]);
         if (j + 1 == n_tiles) umma_commit_elect(&sm.q_empty);  // the unit's last QK^T is issued
         if (j >= 1) issue_pv(g - 1, j == 1);
       }
@@ -270,15 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
       if (a.g.causal) limit = min(limit, t + req.kv_len - req.qo_len + 1);
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < n_tiles; ++j, ++g) {
-        const int st = g & 1;
-        mbar_wait(&sm.s_full[st], (g >> 1) & 1, wc);
+        const int sb = g & 1;
+        mbar_wait(&sm.s_full[sb], (g >> 1) & 1, wc);
         tc_fence_after();
         float sv[kN];
-        tmem_ld32(lane_base + kSCol + st * kN, sv);
-        tmem_ld32(lane_base + kSCol + st * kN + 32, sv + 32);
+        tmem_ld32(lane_base + kSCol + sb * kN, sv);
         tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(&sm.s_free[st]);
+        mbar_arrive(&sm.s_free[sb]);
         const int kv0 = unit.kv_lo + j * kN;
         float mx = -INFINITY;
 #pragma unroll
@@ -323,10 +361,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
               pv[x] = ex2(fmaf(sv[ch * 8 + x], scale, -mu));
               rs += pv[x];
             }
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_addr + row * 128 + ((ch ^ (row & 7)) << 4)),
-                         "r"(pack_bf16x2(pv[0], pv[1])), "r"(pack_bf16x2(pv[2], pv[3])),
-                         "r"(pack_bf16x2(pv[4], pv[5])), "r"(pack_bf16x2(pv[6], pv[7]))
-                         : "memory");
+            st_shared_v4(p_addr + row * 128 + ((ch ^ (row & 7)) << 4), pack_bf16x2(pv[0], pv[1]),
+                         pack_bf16x2(pv[2], pv[3]), pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
           }
           l += rs;
         }
@@ -392,18 +428,39 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
+std::atomic<uint64_t> g_configured{0};  // per-device shared-memory attribute of mla_kernel
+
 }  // namespace
 
 cudaError_t launch_mla(const LaunchGeom& g, const DeviceView& dv, const int32_t* kv_indices, const void* q_nope,
                        const void* q_pe, const void* ckv, const void* kpe, void* o, float* lse,
                        cudaStream_t stream) {
   if (g.num_units == 0 || g.num_ctas == 0) return cudaSuccess;
-  Args a{static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_pe),
-         static_cast<const __nv_bfloat16*>(ckv), static_cast<const __nv_bfloat16*>(kpe), kv_indices,
-         static_cast<__nv_bfloat16*>(o), lse, g, dv};
+  // TMA row coordinates are int32
+  const int64_t q_rows = (int64_t)g.total_q * g.num_qo_heads;
+  if (q_rows <= 0 || q_rows > INT32_MAX) return cudaErrorInvalidValue;
+  // 1. the packed latent rows of every request with queries
+  if (g.packed_rows > 0) {
+    PackArgs pa{static_cast<const __nv_bfloat16*>(ckv), static_cast<const __nv_bfloat16*>(kpe), kv_indices,
+                dv.reqs, dv.kv_row0, static_cast<__nv_bfloat16*>(dv.packed), g.num_reqs, g.page_size,
+                g.page_shift};
+    const dim3 grid((unsigned)((g.max_kv_len + kPackKeys - 1) / kPackKeys), (unsigned)std::min(g.num_reqs, 65535));
+    mla_pack_kernel<<<grid, 256, 0, stream>>>(pa);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // 2. attention over the packed rows
+  Args a{};
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.g = g;
+  a.dv = dv;
+  if (!make_map_2d(&a.tm_q, q_nope, kDc, q_rows, kDc * 2, 64, kRows) ||
+      !make_map_2d(&a.tm_qpe, q_pe, kDr, q_rows, kDr * 2, 64, kRows) ||
+      !make_map_2d(&a.tm_lat, dv.packed, kDqk, std::max(1, g.packed_rows), kDqk * 2, 64, kN))
+    return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
-  static std::atomic<uint64_t> configured{0};
-  cudaError_t e = set_smem_attrs_once((const void*)mla_kernel, (int)smem, configured, false);
+  cudaError_t e = set_smem_attrs_once((const void*)mla_kernel, (int)smem, g_configured, false);
   if (e != cudaSuccess) return e;
   mla_kernel<<<g.num_ctas, kThreads, smem, stream>>>(a);
   return cudaGetLastError();

@@ -73,6 +73,9 @@ struct LaunchGeom {
   int32_t total_q;        // rows of q (tokens)
   int32_t num_ctas;       // CTAs of the main launch (prefill: persistent, one unit list each)
   int32_t kv_layout;      // 0 NHD [page, slot, kv head, D]; 1 HND [page, kv head, slot, D]
+  int32_t packed_rows;    // MLA prefill: rows of the packed latent copy (sum of kv_len of requests with queries)
+  int32_t max_kv_len;     // longest kv_len of the batch
+  int32_t num_reqs;       // requests (batch)
 };
 
 // Device pointers into the workspace after upload.
@@ -84,6 +87,8 @@ struct DeviceView {
   float* part_lse;        // [num_slots, part_rows]
   int* status;            // device status word (0 = ok)
   const int32_t* cta_ptr; // prefill: CTA b runs units [cta_ptr[b], cta_ptr[b + 1])
+  const int32_t* kv_row0; // MLA prefill: first row of each request in the packed latent copy
+  void* packed;           // MLA prefill: packed latent rows [packed_rows][ckv | kpe] bf16
 };
 
 }  // namespace pkv

@@ -95,6 +95,21 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   else if (max_qo <= 1 && group <= kDecodeRows) s.kind = kKindDecode;
   else s.kind = kKindPrefill;
 
+  // MLA prefill streams each request's latent rows from a packed, contiguous
+  // copy (ckv | kpe per key, in key order) that the run builds first; only
+  // requests with queries are packed.
+  int64_t packed_rows = 0;
+  int32_t max_kv = 0;
+  for (int32_t b = 0; b < in.batch; ++b) max_kv = std::max(max_kv, s.reqs[b].kv_len);
+  if (s.kind == kKindMla) {
+    s.kv_row0.assign(in.batch, 0);
+    for (int32_t b = 0; b < in.batch; ++b) {
+      s.kv_row0[b] = (int32_t)std::min<int64_t>(packed_rows, INT32_MAX);
+      if (s.reqs[b].qo_len > 0) packed_rows += s.reqs[b].kv_len;
+    }
+    if (packed_rows > INT32_MAX / 2) { *err = "MLA prefill: more than 2^30 keys in one batch"; return 2; }
+  }
+
   const int32_t num_sms = in.num_sms > 0 ? in.num_sms : 148;
   s.num_sms = num_sms;
   // Rows per work unit: decode packs one token's group of heads into an mma.sync
@@ -261,6 +276,9 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   gm.total_q = in.batch > 0 ? in.qo_indptr[in.batch] : 0;
   gm.num_ctas = num_ctas;
   gm.kv_layout = mla ? 0 : in.kv_layout;  // a latent pool has no head axis: both layouts coincide
+  gm.packed_rows = (int32_t)packed_rows;
+  gm.max_kv_len = max_kv;
+  gm.num_reqs = in.batch;
   *out = std::move(s);
   return 0;
 }

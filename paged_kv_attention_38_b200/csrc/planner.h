@@ -42,6 +42,7 @@ struct Schedule {
   std::vector<WorkUnit> units;
   std::vector<MergeTask> merges;
   std::vector<int32_t> cta_ptr;  // prefill: [num_ctas + 1] offsets of each CTA's units
+  std::vector<int32_t> kv_row0;  // MLA prefill: [batch] first row of each request in the packed latent copy
   int32_t num_slots = 0;
   int32_t kv_chunk = 0;   // chunk used (0 = no split)
   int32_t num_sms = 0;

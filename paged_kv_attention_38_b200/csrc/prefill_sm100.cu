@@ -33,14 +33,13 @@
 // p = 2^(s' - m)). A row's running max m is only moved when the new tile's
 // max exceeds it by more than 8 (p then stays below 2^8 in fp32 / bf16), so O
 // is rescaled in TMEM a few times per row instead of once per tile.
-#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
-#include <cudaTypedefs.h>
 
 #include "launch_util.h"
 #include "pkv_internal.h"
 #include "sm100_ptx.cuh"
+#include "tma_util.h"
 
 namespace pkv {
 
@@ -665,24 +664,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    else
-      cudaGetLastError();
-  }
-  return fn;
-}
-
 // 3-D bf16 tensor [rows][heads][D] (D contiguous), box {64, box_heads, box_rows},
 // 128-byte swizzle, zero fill out of bounds.
 bool make_map(CUtensorMap* m, const void* base, int D, int heads, int64_t rows, int box_heads, int box_rows) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn || rows <= 0) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};

@@ -110,6 +110,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint
       : "memory");
 }
 
+// 2-D tiled bulk tensor load into this CTA's shared memory (x = column,
+// y = row of the tensor map); completion as transaction bytes on `bar`. No multicast.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
 // TMA gather: four rows (r0..r3, any order, out-of-range rows read zeros) of a
 // 2-D tensor, 64 columns from `col`, into four consecutive 128-byte rows of
 // shared memory. The tensor map's box is {64, 1}. No multicast.
