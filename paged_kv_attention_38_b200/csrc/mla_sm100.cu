@@ -31,14 +31,14 @@
 //   SMEM  Q 64 x 576 (72 KB), a 4-stage TMA ring of 32-key latent tiles
 //   (32 x 576, 36 KB: K and V at once, V being the ckv part of the same rows),
 //   P 64 x 32 (in an 8 KB swizzled block).
-// Both MMAs read their operands from shared memory. The tensor core runs a
-// CTA's MMAs in issue order, S(g + 1) then P(g) V(g), so it stays busy while
-// the softmax of a tile runs, and with four stages three tiles are in flight
-// behind the one being consumed. The kernel is persistent: one CTA per SM
-// runs a host-planned list of units, its barrier phases running on across
-// units. Warps: 0-3 softmax and epilogue (lanes 0-15 own S rows and the low O
-// half, lanes 16-31 the high O half of the same rows), 4 TMEM allocator + MMA
-// issuer, 5 TMA producer (one lane).
+// Both MMAs read their operands from shared memory, and two warps issue
+// them: the S MMAs of the next tiles go in while the softmax and the P.V of
+// the current one run, and with four stages three tiles are in flight behind
+// the one being consumed. The kernel is persistent: one CTA per SM runs a
+// host-planned list of units, its barrier phases running on across units.
+// Warps: 0-3 softmax and epilogue (lanes 0-15 own S rows and the low O half,
+// lanes 16-31 the high O half of the same rows), 4 TMEM allocator + S issuer,
+// 5 TMA producer (one lane), 6 P.V issuer.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -63,9 +63,10 @@ constexpr int kBlocks = kDqk / 64;   // 9 column blocks of 64 (128-byte rows)
 constexpr int kQBlockBytes = kRows * 128;  // [64 rows x 64] bf16: 8 KB
 constexpr int kKBlockBytes = kN * 128;     // [32 keys x 64] bf16: 4 KB
 constexpr int kStageBytes = kBlocks * kKBlockBytes;
-constexpr int kThreads = 192;
-constexpr int kMmaWarp = 4;
+constexpr int kThreads = 224;
+constexpr int kMmaWarp = 4;   // TMEM allocator + issuer of the S = Q K^T MMAs
 constexpr int kProdWarp = 5;
+constexpr int kPvWarp = 6;    // issuer of the O += P V MMAs
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol = 256;
 constexpr float kRescaleThreshold = 8.0f;
@@ -230,12 +231,16 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
       for (int k = g - 1; k >= 0 && k >= g - kStages; --k) mbar_drain(&sm.kv_full[k % kStages], (k / kStages) & 1);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ================================================================ MMA issuer
-    // The whole warp runs the loop (waits, descriptor arithmetic); one elected
-    // lane (always lane 0) issues each tcgen05.mma / commit. Issued from a
-    // single divergent lane, each MMA cost about 100 cycles of issue time, more
-    // than its M = 64 execution time.
+  } else if (warp == kMmaWarp || warp == kPvWarp) {
+    // ================================================================ MMA issuers
+    // Two warps issue the tensor-core work: warp kMmaWarp the S = Q K^T MMAs
+    // (36 of N = 32 per tile, each cheap to run but about as costly to issue),
+    // warp kPvWarp the O += P V MMAs. The two streams touch disjoint TMEM (S
+    // buffers / O) and P sits in shared memory, so they need no mutual order;
+    // each stream's own commits keep its barriers exact, and a tile's K/V
+    // stage is released by the P.V commit, which implies its S finished (P
+    // was computed from it). In each warp the whole warp runs the loop (waits,
+    // descriptor arithmetic) and one elected lane issues each instruction.
     constexpr uint32_t idesc_s = idesc_bf16_f32(kRows, kN, false);
     constexpr uint32_t idesc_o = idesc_bf16_f32(kRows, 256, true);
     // Descriptors are built once; another stage, block or K-step only moves the
@@ -245,50 +250,53 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
     const uint64_t dk0 = sdesc_sw128(smem_u32(sm.kv[0]), 16, 1024);
     const uint64_t dv0 = sdesc_sw128(smem_u32(sm.kv[0]), kKBlockBytes, 1024);
     constexpr uint32_t kStageStep = (uint32_t)(kStageBytes >> 4);
-    // O += P V for the CTA's latent tile gg; `first`: the unit's first tile
-    auto issue_pv = [&](int gg, bool first) {
-      const int st = gg % kStages;
-      mbar_wait(&sm.p_full, gg & 1, wc);
-      tc_fence_after();
-#pragma unroll
-      for (int nh = 0; nh < 2; ++nh) {
-        const uint32_t d = tmem + (nh ? (16u << 16) : 0u);
-#pragma unroll
-        for (int kk = 0; kk < kN / 16; ++kk)
-          umma_bf16_ss_elect(d, dp + ((kk * 32) >> 4),
-                             dv0 + st * kStageStep + ((4 * nh * kKBlockBytes + kk * 16 * 128) >> 4), idesc_o,
-                             (!first || kk > 0) ? 1u : 0u);
-      }
-      umma_commit_elect(&sm.o_done);
-      umma_commit_elect(&sm.kv_empty[st]);
-    };
+    const bool s_issuer = warp == kMmaWarp;
     int g = 0;   // latent tiles of this CTA: stage g % kStages, S buffer g & 1 and the per-tile phases
     int uq = 0;  // units with keys: q_full / q_empty / o_final phases
     for (int ui = u_begin; ui < u_end; ++ui) {
       const int n_tiles = tiles_of(a.dv.units[ui]);
       if (n_tiles == 0) continue;
-      mbar_wait(&sm.q_full, uq & 1, wc);
-      for (int j = 0; j < n_tiles; ++j, ++g) {
-        const int st = g % kStages, sb = g & 1;
-        mbar_wait(&sm.kv_full[st], (g / kStages) & 1, wc);
-        if (g >= 2) mbar_wait(&sm.s_free[sb], ((g >> 1) - 1) & 1, wc);
-        tc_fence_after();
+      if (s_issuer) {
+        mbar_wait(&sm.q_full, uq & 1, wc);
+        for (int j = 0; j < n_tiles; ++j, ++g) {
+          const int st = g % kStages, sb = g & 1;
+          mbar_wait(&sm.kv_full[st], (g / kStages) & 1, wc);
+          if (g >= 2) mbar_wait(&sm.s_free[sb], ((g >> 1) - 1) & 1, wc);
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kDqk / 16; ++kk) {
-          const uint32_t oq = ((kk >> 2) * kQBlockBytes + (kk & 3) * 32) >> 4;
-          const uint32_t ok = ((kk >> 2) * kKBlockBytes + (kk & 3) * 32) >> 4;
-          umma_bf16_ss_elect(tmem + kSCol + sb * kN, dq + oq, dk0 + st * kStageStep + ok, idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kDqk / 16; ++kk) {
+            const uint32_t oq = ((kk >> 2) * kQBlockBytes + (kk & 3) * 32) >> 4;
+            const uint32_t ok = ((kk >> 2) * kKBlockBytes + (kk & 3) * 32) >> 4;
+            umma_bf16_ss_elect(tmem + kSCol + sb * kN, dq + oq, dk0 + st * kStageStep + ok, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit_elect(&sm.s_full[sb]);
+          if (j + 1 == n_tiles) umma_commit_elect(&sm.q_empty);  // the unit's last QK^T is issued
         }
-        umma_commit_elect(&sm.s_full[sb]);
-        if (j + 1 == n_tiles) umma_commit_elect(&sm.q_empty);  // the unit's last QK^T is issued
-        if (j >= 1) issue_pv(g - 1, j == 1);
+      } else {
+        // O += P V for each tile of the unit; the first tile overwrites O
+        for (int j = 0; j < n_tiles; ++j, ++g) {
+          const int st = g % kStages;
+          mbar_wait(&sm.p_full, g & 1, wc);
+          tc_fence_after();
+#pragma unroll
+          for (int nh = 0; nh < 2; ++nh) {
+            const uint32_t d = tmem + (nh ? (16u << 16) : 0u);
+#pragma unroll
+            for (int kk = 0; kk < kN / 16; ++kk)
+              umma_bf16_ss_elect(d, dp + ((kk * 32) >> 4),
+                                 dv0 + st * kStageStep + ((4 * nh * kKBlockBytes + kk * 16 * 128) >> 4), idesc_o,
+                                 (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit_elect(&sm.o_done);
+          umma_commit_elect(&sm.kv_empty[st]);
+        }
+        umma_commit_elect(&sm.o_final);
       }
-      issue_pv(g - 1, n_tiles == 1);
-      umma_commit_elect(&sm.o_final);
       ++uq;
     }
-    // no MMA may still run when TMEM is released
-    if (uq > 0) mbar_drain(&sm.o_final, (uq - 1) & 1);
+    // no MMA may still run when TMEM is released (the S stream's last
+    // commits precede the last P.V, which needs every S of its unit)
+    if (!s_issuer && uq > 0) mbar_drain(&sm.o_final, (uq - 1) & 1);
     __syncwarp();
   } else {
     // ================================================================ softmax
