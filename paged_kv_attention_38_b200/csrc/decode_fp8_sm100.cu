@@ -8,17 +8,25 @@
 // and the V scale into the output, so the kernel only has to turn codes into
 // numbers the tensor cores take.
 //
-// The data path is the bf16 decode's, at half the bytes per key: 4 warps
-// stream 64-key tiles of K and V codes (16 KB per stage at head_dim 128)
-// through a 3-stage cp.async ring. Each warp converts its own 16 keys of the
-// tile to f16 (every E4M3 value is exact in f16, one cvt.rn.f16x2.e4m3x2 per
-// pair) into the swizzled rows of one f16 working tile, first K for
-// S = Q K^T, then V into the same rows for O += P V, so only warp barriers
-// separate conversion and use and 64 KB of shared memory lets three CTAs
-// share an SM (the conversion makes the kernel latency-bound with two). Both
-// products run on mma.sync m16n8k16 with f16 operands (Q is rounded to f16
-// once, P is in [0, 1]) and fp32 accumulators; query heads fill the M = 16
-// rows.
+// The data path is the bf16 decode's at half the bytes per key: one CTA per
+// (request, kv head, KV chunk), 4 warps, 64-key tiles of K and V codes
+// (16 KB per stage at head_dim 128) through a 4-stage cp.async ring, three
+// CTAs per SM. Each warp owns 16 keys of a tile and builds its mma.sync
+// m16n8k16 operand fragments straight from the codes in shared memory (one
+// cvt.rn.f16x2.e4m3x2 per pair of codes; every E4M3 value is exact in f16),
+// so every code byte crosses the shared-memory port once. Two permutations
+// make each thread's codes contiguous:
+//   - S = Q K^T sums over the head dimension in any order, so Q and K share
+//     one permutation of it: in k-step kk, lane (g, c) = (lane / 4, lane % 4)
+//     takes the four dims c * D/4 + 4 kk + [0, 4), i.e. the D/4 contiguous
+//     codes [c * D/4, (c + 1) * D/4) of its key row cover all its k-steps.
+//   - In O += P V, column n of n-tile nt stands for dim (D/8) n + nt, so lane
+//     (g, c) reads the D/8 contiguous codes [(D/8) g, (D/8)(g + 1)) of each of
+//     its four key rows; the combine at the end writes each accumulator to
+//     its dim.
+// Q is scaled once per CTA by a power of two that brings its largest |q| to
+// [2^13, 2^14) before the f16 rounding (undone exactly in the score scale), so
+// any finite bf16 query stays in range. P is in [0, 1]; accumulators are fp32.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -32,7 +40,7 @@ namespace pkv {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kTile = kDecodeTileN;  // keys per stage (16 per warp)
 
 struct Args {
@@ -48,22 +56,14 @@ struct Args {
   DeviceView dv;
 };
 
-// Byte offset of 16-byte chunk `ch` (8 f16) of key row `r` in a [kTile x D]
-// f16 tile, chunk index XOR-swizzled by row % 8 (conflict-free ldmatrix).
+// Byte offset of 16-byte chunk `ch` of key row `r` in a [kTile x D] code tile.
+// D = 128: eight chunks per row, XOR-swizzled by row % 8, so that the K reads
+// (eight rows, four chunks) and the V reads (four rows, eight chunks) of a
+// quarter warp hit distinct banks. D = 64: rows of four chunks, unswizzled.
 template <int D>
-__device__ __forceinline__ uint32_t f16_off(int r, int ch) {
-  return (uint32_t)(r * (D * 2) + ((ch ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
+__device__ __forceinline__ uint32_t code_off(int r, int ch) {
+  if constexpr (D == 128) return (uint32_t)(r * D + ((ch ^ (r & 7)) << 4));
+  return (uint32_t)(r * D + (ch << 4));
 }
 
 __device__ __forceinline__ void mma16816_f16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
@@ -87,20 +87,37 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// `n` bytes (16 or 8) of shared memory into words w[0..n/4).
+template <int N>
+__device__ __forceinline__ void ld_codes(uint32_t addr, uint32_t* w) {
+  if constexpr (N == 16) {
+    const uint4 v = ld_shared_v4(addr);
+    w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+  } else if constexpr (N == 32) {
+    const uint4 v0 = ld_shared_v4(addr), v1 = ld_shared_v4(addr + 16);
+    w[0] = v0.x, w[1] = v0.y, w[2] = v0.z, w[3] = v0.w;
+    w[4] = v1.x, w[5] = v1.y, w[6] = v1.z, w[7] = v1.w;
+  } else {
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(addr) : "memory");
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_constant__ Args a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int kCodeTile = kTile * D;       // bytes of one K (or V) code tile
-  constexpr int kChunks = D / 16;            // 16-byte chunks of codes per key row
+  constexpr int kCodeTile = kTile * D;  // bytes of one K (or V) code tile
+  constexpr int kChunks = D / 16;       // 16-byte chunks of codes per key row
+  constexpr int kKSteps = D / 16;       // k-steps of S = Q K^T
+  constexpr int kNTiles = D / 8;        // n-tiles of O += P V
+  constexpr int kKBytes = D / 4;        // contiguous K codes of a lane per key row
+  constexpr int kVBytes = D / 8;        // contiguous V codes of a lane per key row
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int lg = lane >> 2, lc = lane & 3;
   const WorkUnit unit = a.dv.units[blockIdx.x];
   const ReqInfo req = a.dv.reqs[unit.req];
   const int G = a.g.group, Hk = a.g.num_kv_heads, P = a.g.page_size, shift = a.g.page_shift;
   const int n = (unit.kv_hi - unit.kv_lo + kTile - 1) / kTile;
   const uint32_t sbase = smem_u32(smem);
-  // One f16 working tile: each warp converts its 16 K rows, computes S, then
-  // converts its 16 V rows into the same rows for P.V.
-  const uint32_t f16t = sbase + kStages * 2 * kCodeTile;
 
   // All page-table reads of a tile are issued before its copies.
   constexpr int kPerThread = kTile * kChunks / kThreads;
@@ -121,8 +138,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
       const int pos = unit.kv_lo + j * kTile + r;
       const bool ok = page[i] >= 0;
       const size_t off = ok ? (((size_t)page[i] * P + (pos & (P - 1))) * Hk + unit.kv_head) * D + ch * 16 : 0;
-      cp_async_16(kdst + r * D + ch * 16, a.k + off, ok ? 16u : 0u);
-      cp_async_16(vdst + r * D + ch * 16, a.v + off, ok ? 16u : 0u);
+      cp_async_16(kdst + code_off<D>(r, ch), a.k + off, ok ? 16u : 0u);
+      cp_async_16(vdst + code_off<D>(r, ch), a.v + off, ok ? 16u : 0u);
     }
   };
 
@@ -132,33 +149,55 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
     cp_async_commit();
   }
 
-  // Q as f16 mma A fragments: rows = heads of the group (zero past G), k = head_dim.
-  uint32_t qa[D / 16][4];
+  // Q as f16 mma A fragments in the permuted head-dim order: rows = heads of
+  // the group (zero past G); in k-step kk this lane holds dims
+  // lc * D/4 + 4 kk + [0, 2) (a0, a1) and + [2, 4) (a2, a3).
+  uint32_t qa[kKSteps][4];
+  float qscale = 1.f;
   {
-    const int r0 = lane >> 2, kq = (lane & 3) * 2;
     const __nv_bfloat16* qrow = a.q + ((size_t)req.q_start * a.g.num_qo_heads + unit.kv_head * G) * D;
+    float qf[kKSteps][8];
+    float qmax = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      auto ld = [&](int row, int col) -> uint32_t {
-        if (row >= G) return 0u;
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(qrow + (size_t)row * D + col);
-        const float2 f = __bfloat1622float2(b);
-        return pack_f16x2(f.x, f.y);
-      };
-      qa[kk][0] = ld(r0, kk * 16 + kq);
-      qa[kk][1] = ld(r0 + 8, kk * 16 + kq);
-      qa[kk][2] = ld(r0, kk * 16 + kq + 8);
-      qa[kk][3] = ld(r0 + 8, kk * 16 + kq + 8);
+    for (int kk = 0; kk < kKSteps; ++kk) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int row = lg + 8 * h;
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (row < G) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(qrow + (size_t)row * D + lc * kKBytes + 4 * kk);
+          const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+          const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+          f = make_float4(f01.x, f01.y, f23.x, f23.y);
+        }
+        qf[kk][4 * h + 0] = f.x, qf[kk][4 * h + 1] = f.y, qf[kk][4 * h + 2] = f.z, qf[kk][4 * h + 3] = f.w;
+        qmax = fmaxf(qmax, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w))));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+    // power of two bringing qmax to [2^13, 2^14): exact in fp32, undone in the score scale
+    if (qmax > 0.f && qmax < INFINITY) {
+      const int e = (int)((__float_as_uint(qmax) >> 23) & 0xFF) - 127;  // floor(log2 qmax), normal qmax
+      const int se = min(13 - max(e, -126), 127);
+      qscale = __uint_as_float((uint32_t)(127 + se) << 23);
+    }
+#pragma unroll
+    for (int kk = 0; kk < kKSteps; ++kk) {
+      qa[kk][0] = pack_f16x2(qf[kk][0] * qscale, qf[kk][1] * qscale);  // row lg,     dims +0, +1
+      qa[kk][1] = pack_f16x2(qf[kk][4] * qscale, qf[kk][5] * qscale);  // row lg + 8, dims +0, +1
+      qa[kk][2] = pack_f16x2(qf[kk][2] * qscale, qf[kk][3] * qscale);  // row lg,     dims +2, +3
+      qa[kk][3] = pack_f16x2(qf[kk][6] * qscale, qf[kk][7] * qscale);  // row lg + 8, dims +2, +3
     }
   }
 
   const float ks = a.k_scale ? a.k_scale[unit.kv_head] : 1.f;
   const float vs = a.v_scale ? a.v_scale[unit.kv_head] : 1.f;
-  const float scale = a.g.sm_scale_log2 * ks;
-  float o_acc[D / 8][4];
+  const float scale = a.g.sm_scale_log2 * ks / qscale;
+  float o_acc[kNTiles][4];
 #pragma unroll
-  for (int i = 0; i < D / 8; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows lane/4 and lane/4 + 8
+  for (int i = 0; i < kNTiles; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows lg and lg + 8
 
   for (int j = 0; j < n; ++j) {
     cp_async_wait<kStages - 2>();
@@ -166,38 +205,28 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
     if (j + kStages - 1 < n) load_tile(j + kStages - 1, (j + kStages - 1) % kStages);
     cp_async_commit();
 
-    // this warp's 16 keys of the tile: codes -> f16 rows (t = 0: K, t = 1: V)
-    const uint32_t kcode = sbase + (j % kStages) * 2 * kCodeTile;
-    auto convert = [&](int t) {
-      const uint32_t src = kcode + t * kCodeTile;
-#pragma unroll
-      for (int c = lane; c < 16 * kChunks; c += 32) {
-        const int r = warp * 16 + c / kChunks, ch = c % kChunks;
-        const uint4 w = ld_shared_v4(src + r * D + ch * 16);
-        st_shared_v4(f16t + f16_off<D>(r, 2 * ch), e4m3x2_to_f16x2(w.x), e4m3x2_to_f16x2(w.x >> 16),
-                     e4m3x2_to_f16x2(w.y), e4m3x2_to_f16x2(w.y >> 16));
-        st_shared_v4(f16t + f16_off<D>(r, 2 * ch + 1), e4m3x2_to_f16x2(w.z), e4m3x2_to_f16x2(w.z >> 16),
-                     e4m3x2_to_f16x2(w.w), e4m3x2_to_f16x2(w.w >> 16));
-      }
-      __syncwarp();
-    };
-    convert(0);
-
-    // S[16 x 16] = Q . K^T for this warp's 16 keys
+    const uint32_t kst = sbase + (j % kStages) * 2 * kCodeTile;
+    const uint32_t vst = kst + kCodeTile;
+    const int r0 = warp * 16;  // this warp's 16 keys of the tile
+    // S[16 x 16] = Q . K^T: n-tile t holds keys r0 + 8t + [0, 8); this lane's
+    // B fragments come from key r0 + 8t + lg, codes [lc * D/4, +D/4)
     float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    {
-      const int mi = lane >> 3;
-      const int row = warp * 16 + (lane & 7) + (mi >> 1) * 8;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(f16t + f16_off<D>(row, kk * 2 + (mi & 1)), b0, b1, b2, b3);
-        mma16816_f16(s[0], qa[kk], b0, b1);
-        mma16816_f16(s[1], qa[kk], b2, b3);
+    for (int t = 0; t < 2; ++t) {
+      const int r = r0 + 8 * t + lg;
+      uint32_t w[kKBytes / 4];
+      if constexpr (D == 128) {
+        ld_codes<16>(kst + code_off<D>(r, 2 * lc), w);
+        ld_codes<16>(kst + code_off<D>(r, 2 * lc + 1), w + 4);
+      } else {
+        ld_codes<16>(kst + code_off<D>(r, lc), w);
       }
+#pragma unroll
+      for (int kk = 0; kk < kKSteps; ++kk)
+        mma16816_f16(s[t], qa[kk], e4m3x2_to_f16x2(w[kk]), e4m3x2_to_f16x2(w[kk] >> 16));
     }
     // mask keys past the unit's end, scale into the base-2 domain
-    const int key0 = unit.kv_lo + j * kTile + warp * 16 + (lane & 3) * 2;
+    const int key0 = unit.kv_lo + j * kTile + r0 + lc * 2;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
@@ -230,36 +259,50 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
     l0 = l0 * a0 + rs0;
     l1 = l1 * a1 + rs1;
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
+    for (int i = 0; i < kNTiles; ++i) {
       o_acc[i][0] *= a0;
       o_acc[i][1] *= a0;
       o_acc[i][2] *= a1;
       o_acc[i][3] *= a1;
     }
-    __syncwarp();  // every lane's K fragments are read before V overwrites the rows
-    convert(1);
+    // P as the A fragment: keys r0 + 2lc, +1 (a0, a1) and r0 + 8 + 2lc, +1 (a2, a3)
     uint32_t pa[4];
     pa[0] = pack_f16x2(s[0][0], s[0][1]);
     pa[1] = pack_f16x2(s[0][2], s[0][3]);
     pa[2] = pack_f16x2(s[1][0], s[1][1]);
     pa[3] = pack_f16x2(s[1][2], s[1][3]);
+    // O += P V: the B fragment of n-tile nt pairs the codes of keys (2lc, 2lc + 1)
+    // and (2lc + 8, 2lc + 9) at dim (D/8) lg + nt, byte nt of this lane's run
     {
-      const int mi = lane >> 3;
-      const int row = warp * 16 + (lane & 7) + (mi & 1) * 8;
+      uint32_t va[kVBytes / 4], vb[kVBytes / 4], vc[kVBytes / 4], vd[kVBytes / 4];
+      const int rk = r0 + 2 * lc;
+      if constexpr (D == 128) {
+        ld_codes<16>(vst + code_off<D>(rk, lg), va);
+        ld_codes<16>(vst + code_off<D>(rk + 1, lg), vb);
+        ld_codes<16>(vst + code_off<D>(rk + 8, lg), vc);
+        ld_codes<16>(vst + code_off<D>(rk + 9, lg), vd);
+      } else {
+        ld_codes<8>(vst + rk * D + lg * kVBytes, va);
+        ld_codes<8>(vst + (rk + 1) * D + lg * kVBytes, vb);
+        ld_codes<8>(vst + (rk + 8) * D + lg * kVBytes, vc);
+        ld_codes<8>(vst + (rk + 9) * D + lg * kVBytes, vd);
+      }
 #pragma unroll
-      for (int np = 0; np < D / 16; ++np) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(f16t + f16_off<D>(row, np * 2 + (mi >> 1)), b0, b1, b2, b3);
-        mma16816_f16(o_acc[np * 2], pa, b0, b1);
-        mma16816_f16(o_acc[np * 2 + 1], pa, b2, b3);
+      for (int wi = 0; wi < kVBytes / 4; ++wi) {
+        const uint32_t lo01 = __byte_perm(va[wi], vb[wi], 0x5140), hi01 = __byte_perm(va[wi], vb[wi], 0x7362);
+        const uint32_t lo89 = __byte_perm(vc[wi], vd[wi], 0x5140), hi89 = __byte_perm(vc[wi], vd[wi], 0x7362);
+        mma16816_f16(o_acc[4 * wi + 0], pa, e4m3x2_to_f16x2(lo01), e4m3x2_to_f16x2(lo89));
+        mma16816_f16(o_acc[4 * wi + 1], pa, e4m3x2_to_f16x2(lo01 >> 16), e4m3x2_to_f16x2(lo89 >> 16));
+        mma16816_f16(o_acc[4 * wi + 2], pa, e4m3x2_to_f16x2(hi01), e4m3x2_to_f16x2(hi89));
+        mma16816_f16(o_acc[4 * wi + 3], pa, e4m3x2_to_f16x2(hi01 >> 16), e4m3x2_to_f16x2(hi89 >> 16));
       }
     }
-    __syncwarp();  // the next tile's conversion overwrites this warp's f16 rows
   }
   cp_async_wait<0>();
   __syncthreads();
 
-  // ---- combine the 4 warps' states through shared memory
+  // ---- combine the 4 warps' states through shared memory; accumulator
+  // (nt, column 2lc + x) of this lane is dim (D/8)(2lc + x) + nt
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
@@ -268,20 +311,20 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
   float* sm_m = so + 4 * 16 * D;                         // [4][16]
   float* sm_l = sm_m + 4 * 16;                           // [4][16]
   {
-    const int r0 = lane >> 2, c0 = (lane & 3) * 2;
     float* ow = so + warp * 16 * D;
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      ow[r0 * D + i * 8 + c0] = o_acc[i][0];
-      ow[r0 * D + i * 8 + c0 + 1] = o_acc[i][1];
-      ow[(r0 + 8) * D + i * 8 + c0] = o_acc[i][2];
-      ow[(r0 + 8) * D + i * 8 + c0 + 1] = o_acc[i][3];
+    for (int nt = 0; nt < kNTiles; ++nt) {
+      const int d0 = kVBytes * (2 * lc) + nt, d1 = kVBytes * (2 * lc + 1) + nt;
+      ow[lg * D + d0] = o_acc[nt][0];
+      ow[lg * D + d1] = o_acc[nt][1];
+      ow[(lg + 8) * D + d0] = o_acc[nt][2];
+      ow[(lg + 8) * D + d1] = o_acc[nt][3];
     }
-    if ((lane & 3) == 0) {
-      sm_m[warp * 16 + r0] = m0;
-      sm_m[warp * 16 + r0 + 8] = m1;
-      sm_l[warp * 16 + r0] = l0;
-      sm_l[warp * 16 + r0 + 8] = l1;
+    if (lc == 0) {
+      sm_m[warp * 16 + lg] = m0;
+      sm_m[warp * 16 + lg + 8] = m1;
+      sm_l[warp * 16 + lg] = l0;
+      sm_l[warp * 16 + lg + 8] = l1;
     }
   }
   __syncthreads();
@@ -314,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
 
 template <int D>
 cudaError_t launch(const Args& a, cudaStream_t stream) {
-  const size_t pipe = (size_t)kStages * 2 * kTile * D + (size_t)kTile * D * 2;
+  const size_t pipe = (size_t)kStages * 2 * kTile * D;
   const size_t comb = (size_t)4 * 16 * D * 4 + 2 * 4 * 16 * 4;
   const size_t smem = pipe > comb ? pipe : comb;
   auto kern = decode_fp8_kernel<D>;

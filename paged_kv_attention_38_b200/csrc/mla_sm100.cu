@@ -213,6 +213,14 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
           tma_load_2d(smem_u32(sm.q) + blk * kQBlockBytes, &a.tm_q, &sm.q_full, blk * 64, qrow);
         tma_load_2d(smem_u32(sm.q) + (kBlocks - 1) * kQBlockBytes, &a.tm_qpe, &sm.q_full, 0, qrow);
         ++uq;
+        // warm L2 with the next unit's Q so its load at the unit boundary is short
+        if (ui + 1 < u_end) {
+          const WorkUnit nu = a.dv.units[ui + 1];
+          const int nrow = a.dv.reqs[nu.req].q_start * H + nu.row0;
+#pragma unroll
+          for (int blk = 0; blk < kBlocks - 1; ++blk) tma_prefetch_l2_2d(&a.tm_q, blk * 64, nrow);
+          tma_prefetch_l2_2d(&a.tm_qpe, 0, nrow);
+        }
         const int krow0 = a.dv.kv_row0[unit.req] + unit.kv_lo;
         for (int j = 0; j < n_tiles; ++j, ++g) {
           const int st = g % kStages;

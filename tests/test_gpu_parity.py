@@ -295,6 +295,27 @@ def test_fp8_kv_decode_unit_scales():
     assert_parity(o, lse, *oracle_fp8(p, k_scale=False, v_scale=False), what="fp8 decode unit scales")
 
 
+@pytest.mark.parametrize("qmul", [1e5, 1e-6])
+def test_fp8_kv_decode_query_range(qmul):
+    """Queries far outside the f16 range (|q| up to ~5e5, where f16 overflows) and
+    deep in its subnormals (|q| ~ 1e-6): the kernel scales Q by a power of two
+    before the f16 rounding. O is checked at the stated tolerance; with |q| ~ 1e5
+    the LSE is ~1e5 and fp32 resolves it to ~1e-2, so there it is checked to
+    1e-6 relative."""
+    p = W.make_fp8_kv_problem("fp8range", [1, 1, 1], [300, 77, 1000], num_qo_heads=16, num_kv_heads=2,
+                              head_dim=128, page_size=16, seed=int(qmul < 1) + 41)
+    p.q = (p.q.float() * qmul).to(torch.bfloat16)
+    o, lse, _ = gpu_run_fp8(p)
+    o_ref, l_ref = oracle_fp8(p)
+    if qmul > 1:
+        assert np.all(np.isfinite(lse.cpu().numpy()))
+        err = np.abs(lse.cpu().double().numpy() - l_ref)
+        assert np.all(err <= 1e-3 + 1e-6 * np.abs(l_ref)), err.max()
+        assert_parity(o, np.nan_to_num(l_ref), o_ref, np.nan_to_num(l_ref), what=f"fp8 q x {qmul}")
+    else:
+        assert_parity(o, lse, o_ref, l_ref, what=f"fp8 q x {qmul}")
+
+
 def test_fp8_kv_rejects_prefill_plan():
     p = W.make_fp8_kv_problem("fp8pre", [4, 2], [40, 9], num_qo_heads=4, num_kv_heads=2, head_dim=128,
                               page_size=16, seed=4)
