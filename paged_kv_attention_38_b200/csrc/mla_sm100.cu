@@ -271,11 +271,16 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
           mbar_wait(&sm.kv_full[st], (g / kStages) & 1, wc);
           if (g >= 2) mbar_wait(&sm.s_free[sb], ((g >> 1) - 1) & 1, wc);
           tc_fence_after();
+          const uint64_t dk = dk0 + st * kStageStep;
 #pragma unroll
-          for (int kk = 0; kk < kDqk / 16; ++kk) {
-            const uint32_t oq = ((kk >> 2) * kQBlockBytes + (kk & 3) * 32) >> 4;
-            const uint32_t ok = ((kk >> 2) * kKBlockBytes + (kk & 3) * 32) >> 4;
-            umma_bf16_ss_elect(tmem + kSCol + sb * kN, dq + oq, dk0 + st * kStageStep + ok, idesc_s, kk > 0 ? 1u : 0u);
+          for (int b = 0; b < kBlocks; ++b) {  // four K-steps of one 64-column block per elect
+            uint64_t da[4], db[4];
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              da[k4] = dq + ((b * kQBlockBytes + k4 * 32) >> 4);
+              db[k4] = dk + ((b * kKBlockBytes + k4 * 32) >> 4);
+            }
+            umma4_bf16_ss_elect(tmem + kSCol + sb * kN, da, db, idesc_s, b > 0 ? 1u : 0u);
           }
           umma_commit_elect(&sm.s_full[sb]);
           if (j + 1 == n_tiles) umma_commit_elect(&sm.q_empty);  // the unit's last QK^T is issued
