@@ -355,9 +355,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     auto issue_s = [&](int i, int item) {
       const uint64_t bq = dq0 + i * kQStep, bk = dk0 + (item & (kSlots - 1)) * kSlotStep;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
-        umma_bf16_ss_elect(tmem + i * kBlockN, bq + off, bk + off, idesc_s, kk > 0 ? 1u : 0u);
+      for (int k0 = 0; k0 < D / 16; k0 += 4) {  // the four K-steps of a 64-column block per elect
+        uint64_t da[4], db[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const uint32_t off = (((k0 + x) >> 2) * (kTileM * 128) + ((k0 + x) & 3) * 32) >> 4;
+          da[x] = bq + off;
+          db[x] = bk + off;
+        }
+        umma4_bf16_ss_elect(tmem + i * kBlockN, da, db, idesc_s, k0 > 0 ? 1u : 0u);
       }
       umma_commit_elect(&sm.s_full[i]);
     };
@@ -365,10 +371,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // `first`: the unit's first KV tile, which overwrites O_i.
     auto issue_pv_half = [&](int i, int item, int h, bool first) {
       const uint64_t bv = dv0 + (item & (kSlots - 1)) * kSlotStep;
+      uint32_t ta[4];
+      uint64_t db[4];
 #pragma unroll
-      for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
-        umma_bf16_ts_elect(tmem + 256 + i * 128, tmem + i * kBlockN + kk * 8, bv + ((kk * 16 * 128) >> 4),
-                           idesc_o, (!first || kk > 0) ? 1u : 0u);
+      for (int x = 0; x < 4; ++x) {
+        const int kk = 4 * h + x;
+        ta[x] = tmem + i * kBlockN + kk * 8;
+        db[x] = bv + ((kk * 16 * 128) >> 4);
+      }
+      umma4_bf16_ts_elect(tmem + 256 + i * 128, ta, db, idesc_o, (!first || h > 0) ? 1u : 0u);
     };
     int jt = 0;  // KV tiles done by this CTA (all units): s_full / p_half phases
     int uq = 0;  // units with keys: q_full / q_empty / o_final phases

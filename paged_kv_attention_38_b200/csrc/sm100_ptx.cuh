@@ -268,6 +268,24 @@ __device__ __forceinline__ void umma4_bf16_ss_elect(uint32_t d_tmem, const uint6
       : "memory");
 }
 
+// Four TS MMAs (A from tensor memory) into one accumulator under one
+// elect.sync: A at TMEM addresses a[i], B descriptors b[i]; the first
+// accumulates iff `accumulate`, the other three always do.
+__device__ __forceinline__ void umma4_bf16_ts_elect(uint32_t d_tmem, const uint32_t* a, const uint64_t* b, uint32_t idesc,
+                                                    uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %9, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %9, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %9, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %9, 1;\n\t}" ::"r"(d_tmem),
+      "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc),
+      "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void umma_commit_elect(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
