@@ -54,12 +54,6 @@ constexpr int kProdWarp0 = 9;
 constexpr int kProdThreads = 96;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
-// Columns c with (c % 8) < kPolyPer8 take 2^x from the FMA-pipe polynomial,
-// the rest from MUFU ex2: the split that balances the two pipes.
-#ifndef PKV_POLY_PER8
-#define PKV_POLY_PER8 0
-#endif
-constexpr int kPolyPer8 = PKV_POLY_PER8;
 constexpr int kRegsSupport = 96;
 constexpr int kRegsSoftmax = 200;
 static_assert(128 * kRegsSupport + 256 * kRegsSoftmax <= kThreads * 168, "register split exceeds the launch budget");
@@ -105,7 +99,7 @@ struct Args {
   LaunchGeom g;
   DeviceView dv;
   int32_t q_tma;      // Q tiles by TMA (group divides 128) or by cp.async
-  int32_t kv_tma;     // K/V pages by TMA (page_size >= 8) or by cp.async rows
+  int32_t kv_tma;     // K/V pages by TMA (page_size >= 8; the kRows = false instance) or by cp.async rows
   int32_t oob_row;    // a pool row index past the end: TMA zero-fills it
 };
 
@@ -134,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     mbar_init(&sm.q_full, a.q_tma ? 1 : kProdThreads);
     mbar_init(&sm.q_empty, 1);
     for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&sm.full[s], (!kRows && a.kv_tma) ? 1 : kProdThreads);
+      mbar_init(&sm.full[s], kRows ? kProdThreads : 1);
       mbar_init(&sm.empty[s], 1);
     }
     for (int i = 0; i < kTiles; ++i) {
@@ -169,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const int P = a.g.page_size, shift = a.g.page_shift, Hk = a.g.num_kv_heads;
     if (pt == 0) {
       if (a.q_tma) tma_prefetch_desc(&a.tm_q);
-      if (!kRows && a.kv_tma) {
+      if constexpr (!kRows) {
         tma_prefetch_desc(&a.tm_k);
         tma_prefetch_desc(&a.tm_v);
       }
@@ -226,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const int j = k >> 1;
         const bool is_v = k & 1;
         const int pos0 = unit.kv_lo + j * kBlockN;
-        if (!kRows && a.kv_tma) {
+        if constexpr (!kRows) {
           if (pt == 0) {
             if (kc >= kSlots) mbar_wait(&sm.empty[slot], ((kc >> 2) - 1) & 1, wc);
             mbar_arrive_expect_tx(&sm.full[slot], kBlockN * D * 2);
@@ -281,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             }
             named_bar_sync(1, kProdThreads);
           }
-          if (kRows) {
+          {
             // thread pt copies 16-byte column ch of rows r0, r0 + kRowStep, ...:
             // the source row is read once per row and the column offset is fixed.
             const __nv_bfloat16* base = (is_v ? a.v : a.k) + unit.kv_head * D;
@@ -301,22 +295,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
               }
               cp_async_16(dst + r * 128 + (col_off ^ ((r & 7) << 4)), g, src >= 0 ? 16u : 0u);
             }
-          } else {
-            // (the page-gather instance never runs this; it is kept so that its
-            // register allocation matches the measured fast build)
-            const __nv_bfloat16* base = is_v ? a.v : a.k;
-            const uint32_t dst = smem_u32(sm.kv[slot]);
-            for (int c = pt; c < kBlockN * kChunks; c += kProdThreads) {
-              const int r = c / kChunks, ch = c % kChunks;
-              const int src = sm.rowsrc[r];
-              const __nv_bfloat16* g;
-              if constexpr (kHnd)
-                g = src >= 0 ? base + (((size_t)(src >> shift) * Hk + unit.kv_head) * P + (src & (P - 1))) * D + ch * 8
-                             : base;
-              else
-                g = src >= 0 ? base + ((size_t)src * Hk + unit.kv_head) * D + ch * 8 : base;
-              cp_async_16(dst + tile_off(r, ch), g, src >= 0 ? 16u : 0u);
-            }
           }
           cp_async_arrive_noinc(&sm.full[slot]);
         }
@@ -328,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     // was consumed before its slot was refilled).
     if (pt == 0) {
       if (a.q_tma && uq > 0) mbar_drain(&sm.q_full, (uq - 1) & 1);
-      if (!kRows && a.kv_tma)
+      if constexpr (!kRows)
         for (int k = kc - 1; k >= 0 && k >= kc - kSlots; --k) mbar_drain(&sm.full[k & (kSlots - 1)], (k >> 2) & 1);
     }
   } else if (warp == kMmaWarp) {
@@ -503,16 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             const int c = h * 64 + 2 * e;
             const float2 x = ffma2(make_float2(sv[c], sv[c + 1]), scale2, nmu2);
             float2 pp;
-            if (kPolyPer8 > 0 && ((2 * e) & 7) < kPolyPer8) {
-              pp = exp2_poly2(x);
-              if (!whole) {
-                if (sv[c] == -INFINITY) pp.x = 0.f;
-                if (sv[c + 1] == -INFINITY) pp.y = 0.f;
-              }
-            } else {
-              pp.x = ex2(x.x);
-              pp.y = ex2(x.y);
-            }
+            pp.x = ex2(x.x);
+            pp.y = ex2(x.y);
             if (e & 1) rs2b = fadd2(rs2b, pp);
             else rs2a = fadd2(rs2a, pp);
             pw[e] = pack_bf16x2(pp.x, pp.y);

@@ -390,26 +390,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for use beside ex2 (the MUFU pipe is the softmax's
-// bottleneck). Round-to-nearest range reduction x = j + f, f in [-1/2, 1/2],
-// through the 1.5 * 2^23 shifter (j lands in the low mantissa bits of t), then
-// a degree-3 polynomial for 2^f and j added into the exponent field.
-// Coefficients: our own minimax fit of 2^f on [-1/2, 1/2] in relative error
-// (Lawson's iteratively reweighted least squares, then rounded to fp32);
-// max relative error 7.5e-5, far below the bf16 rounding P gets next.
-// Inputs below -126 are clamped (the result is then ~2^-126, i.e. 0 for P).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float shifter = 12582912.0f;  // 1.5 * 2^23
-  const float t = x + shifter;
-  const float j = t - shifter;
-  const float f = x - j;
-  float p = fmaf(0.0551716685f, f, 0.2426111400f);
-  p = fmaf(p, f, 0.6932609677f);
-  p = fmaf(p, f, 0.9999280572f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Packed fp32 pair arithmetic (one instruction for two lanes of work).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   uint64_t d;
@@ -432,21 +412,6 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   float2 r;
   asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
   return r;
-}
-
-// Two lanes of exp2_poly with packed fp32 arithmetic.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 sh = make_float2(12582912.0f, 12582912.0f);
-  const float2 t = fadd2(x, sh);
-  const float2 j = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = ffma2(j, make_float2(-1.f, -1.f), x);
-  float2 p = ffma2(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.2426111400f, 0.2426111400f));
-  p = ffma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
-  p = ffma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
