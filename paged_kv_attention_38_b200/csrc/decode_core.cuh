@@ -206,12 +206,16 @@ __device__ __forceinline__ void attend(uint8_t* smem, const Job& jb) {
     }
     l0 = l0 * a0 + rs0;
     l1 = l1 * a1 + rs1;
+    // O *= alpha only when some row of the warp moved its max (after the first
+    // tiles the max rarely moves; the result is the same either way)
+    if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      o_acc[i][0] *= a0;
-      o_acc[i][1] *= a0;
-      o_acc[i][2] *= a1;
-      o_acc[i][3] *= a1;
+      for (int i = 0; i < D / 8; ++i) {
+        o_acc[i][0] *= a0;
+        o_acc[i][1] *= a0;
+        o_acc[i][2] *= a1;
+        o_acc[i][3] *= a1;
+      }
     }
     uint32_t pa[4];
     pa[0] = pack_bf16x2(s[0][0], s[0][1]);

@@ -74,12 +74,15 @@ __device__ __forceinline__ void mma16816_f16(float* d, const uint32_t* a, uint32
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Two E4M3 codes (low byte = lower element) -> f16x2 (low half = lower element).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-  uint32_t out;
-  const unsigned short in = (unsigned short)two_codes;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(out) : "h"(in));
-  return out;
+// Four E4M3 codes (bytes 0..3 of w) -> two f16x2: lo = (byte 0, byte 1),
+// hi = (byte 2, byte 3).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -222,8 +225,11 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
         ld_codes<16>(kst + code_off<D>(r, lc), w);
       }
 #pragma unroll
-      for (int kk = 0; kk < kKSteps; ++kk)
-        mma16816_f16(s[t], qa[kk], e4m3x2_to_f16x2(w[kk]), e4m3x2_to_f16x2(w[kk] >> 16));
+      for (int kk = 0; kk < kKSteps; ++kk) {
+        uint32_t b0, b1;
+        e4m3x4_to_f16x2x2(w[kk], b0, b1);
+        mma16816_f16(s[t], qa[kk], b0, b1);
+      }
     }
     // mask keys past the unit's end, scale into the base-2 domain
     const int key0 = unit.kv_lo + j * kTile + r0 + lc * 2;
@@ -258,12 +264,16 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
     }
     l0 = l0 * a0 + rs0;
     l1 = l1 * a1 + rs1;
+    // O *= alpha only when some row of the warp moved its max (after the first
+    // tiles the max rarely moves; the result is the same either way)
+    if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
 #pragma unroll
-    for (int i = 0; i < kNTiles; ++i) {
-      o_acc[i][0] *= a0;
-      o_acc[i][1] *= a0;
-      o_acc[i][2] *= a1;
-      o_acc[i][3] *= a1;
+      for (int i = 0; i < kNTiles; ++i) {
+        o_acc[i][0] *= a0;
+        o_acc[i][1] *= a0;
+        o_acc[i][2] *= a1;
+        o_acc[i][3] *= a1;
+      }
     }
     // P as the A fragment: keys r0 + 2lc, +1 (a0, a1) and r0 + 8 + 2lc, +1 (a2, a3)
     uint32_t pa[4];
@@ -289,12 +299,13 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
       }
 #pragma unroll
       for (int wi = 0; wi < kVBytes / 4; ++wi) {
-        const uint32_t lo01 = __byte_perm(va[wi], vb[wi], 0x5140), hi01 = __byte_perm(va[wi], vb[wi], 0x7362);
-        const uint32_t lo89 = __byte_perm(vc[wi], vd[wi], 0x5140), hi89 = __byte_perm(vc[wi], vd[wi], 0x7362);
-        mma16816_f16(o_acc[4 * wi + 0], pa, e4m3x2_to_f16x2(lo01), e4m3x2_to_f16x2(lo89));
-        mma16816_f16(o_acc[4 * wi + 1], pa, e4m3x2_to_f16x2(lo01 >> 16), e4m3x2_to_f16x2(lo89 >> 16));
-        mma16816_f16(o_acc[4 * wi + 2], pa, e4m3x2_to_f16x2(hi01), e4m3x2_to_f16x2(hi89));
-        mma16816_f16(o_acc[4 * wi + 3], pa, e4m3x2_to_f16x2(hi01 >> 16), e4m3x2_to_f16x2(hi89 >> 16));
+        uint32_t b01[4], b89[4];
+        e4m3x4_to_f16x2x2(__byte_perm(va[wi], vb[wi], 0x5140), b01[0], b01[1]);
+        e4m3x4_to_f16x2x2(__byte_perm(va[wi], vb[wi], 0x7362), b01[2], b01[3]);
+        e4m3x4_to_f16x2x2(__byte_perm(vc[wi], vd[wi], 0x5140), b89[0], b89[1]);
+        e4m3x4_to_f16x2x2(__byte_perm(vc[wi], vd[wi], 0x7362), b89[2], b89[3]);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) mma16816_f16(o_acc[4 * wi + x], pa, b01[x], b89[x]);
       }
     }
   }
