@@ -157,9 +157,11 @@ PKV_API pkv_status pkv_run_mla(const pkv_plan* plan, const void* q_nope, const v
  * pkv_run's attention over those values: q, o, lse as there. The plan must be
  * a decode plan from pkv_plan_create (every qo_len <= 1, group <= 16) with the
  * NHD layout and head_dim 64 or 128; anything else returns PKV_EUNSUPPORTED.
- * On the device Q is rounded to f16 (|q| must lie within the f16 range) and P
- * to f16, every code converts exactly to f16, and O and the LSE accumulate in
- * fp32; NaN codes propagate. Pointers 16-byte aligned; num_pages as in
+ * On the device each CTA scales its Q rows by a power of two that brings their
+ * largest |q| to [2^13, 2^14) (undone exactly in the score scale) and rounds
+ * them to f16, so any finite bf16 q is accepted; P is rounded to f16, every
+ * code converts exactly to f16, and O and the LSE accumulate in fp32; NaN
+ * codes propagate. Pointers 16-byte aligned; num_pages as in
  * pkv_run. Never allocates, never synchronises; the split-KV merge runs on the
  * same stream. */
 PKV_API pkv_status pkv_run_fp8_kv(const pkv_plan* plan, const void* q, const void* k_codes, const void* v_codes,
