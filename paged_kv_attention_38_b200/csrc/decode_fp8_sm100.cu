@@ -122,18 +122,20 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
   const int n = (unit.kv_hi - unit.kv_lo + kTile - 1) / kTile;
   const uint32_t sbase = smem_u32(smem);
 
-  // All page-table reads of a tile are issued before its copies.
+  // Page ids are read one tile ahead of the copies that use them, during the
+  // previous tile's math, so no warp waits a global-memory latency per tile.
   constexpr int kPerThread = kTile * kChunks / kThreads;
   static_assert(kTile * kChunks % kThreads == 0, "whole copies per thread");
-  auto load_tile = [&](int j, int stage) {
-    const uint32_t kdst = sbase + stage * 2 * kCodeTile;
-    const uint32_t vdst = kdst + kCodeTile;
-    int page[kPerThread];
+  auto fetch_pages = [&](int j, int* page) {
 #pragma unroll
     for (int i = 0; i < kPerThread; ++i) {
       const int pos = unit.kv_lo + j * kTile + (tid + i * kThreads) / kChunks;
       page[i] = pos < unit.kv_hi ? __ldg(a.kv_indices + req.page0 + (pos >> shift)) : -1;
     }
+  };
+  auto load_tile = [&](int j, int stage, const int* page) {
+    const uint32_t kdst = sbase + stage * 2 * kCodeTile;
+    const uint32_t vdst = kdst + kCodeTile;
 #pragma unroll
     for (int i = 0; i < kPerThread; ++i) {
       const int c = tid + i * kThreads;
@@ -146,11 +148,16 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
     }
   };
 
+  int page_next[kPerThread];  // ids of tile (j + kStages - 1), read during tile j - 1
 #pragma unroll
   for (int s = 0; s < kStages - 1; ++s) {
-    if (s < n) load_tile(s, s);
+    if (s < n) {
+      fetch_pages(s, page_next);
+      load_tile(s, s, page_next);
+    }
     cp_async_commit();
   }
+  if (kStages - 1 < n) fetch_pages(kStages - 1, page_next);
 
   // Q as f16 mma A fragments in the permuted head-dim order: rows = heads of
   // the group (zero past G); in k-step kk this lane holds dims
@@ -205,8 +212,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
   for (int j = 0; j < n; ++j) {
     cp_async_wait<kStages - 2>();
     __syncthreads();
-    if (j + kStages - 1 < n) load_tile(j + kStages - 1, (j + kStages - 1) % kStages);
+    if (j + kStages - 1 < n) load_tile(j + kStages - 1, (j + kStages - 1) % kStages, page_next);
     cp_async_commit();
+    if (j + kStages < n) fetch_pages(j + kStages, page_next);
 
     const uint32_t kst = sbase + (j % kStages) * 2 * kCodeTile;
     const uint32_t vst = kst + kCodeTile;

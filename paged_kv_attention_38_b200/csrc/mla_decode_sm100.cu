@@ -114,17 +114,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) mla_decode_kernel(const 
   // latent rows of tile j -> stage: 64 ckv chunks then 8 kpe chunks per key.
   // Four threads per key: one page-table read per thread, then 18 copies
   // (chunks q, q + 4, ...: each warp instruction covers 64 contiguous bytes of
-  // 8 rows). Looking the page up inside the copy loop would serialise a
-  // global read before every copy (the copies are ordered memory operations).
+  // 8 rows). The page id of a tile is read one tile ahead, during the previous
+  // tile's math: read inside the copy loop it would serialise a global read
+  // before every copy (the copies are ordered memory operations), and read
+  // just before the loop it would stall the warp one memory latency a tile.
   static_assert(kThreads == 4 * kKeys, "four threads per key row");
-  auto load_tile = [&](int j, int stage) {
+  auto fetch_slot = [&](int j) -> long long {
+    const int pos = unit.kv_lo + j * kKeys + (tid >> 2);
+    if (pos >= unit.kv_hi) return -1;
+    return (long long)__ldg(a.kv_indices + req.page0 + (pos >> shift)) * P + (pos & (P - 1));
+  };
+  auto load_tile = [&](int stage, long long slot_or_neg) {
     const uint32_t cdst = sbase + kOffStage + stage * kStageBytes;
     const uint32_t kdst = cdst + kCkvBytes;
     const int r = tid >> 2, q = tid & 3;
-    const int pos = unit.kv_lo + j * kKeys + r;
-    const bool ok = pos < unit.kv_hi;
-    size_t slot = 0;
-    if (ok) slot = (size_t)__ldg(a.kv_indices + req.page0 + (pos >> shift)) * P + (pos & (P - 1));
+    const bool ok = slot_or_neg >= 0;
+    const size_t slot = ok ? (size_t)slot_or_neg : 0;
     const __nv_bfloat16* csrc = a.ckv + slot * kDc;
     const __nv_bfloat16* ksrc = a.kpe + slot * kDr;
 #pragma unroll
@@ -145,9 +150,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) mla_decode_kernel(const 
   }
 #pragma unroll
   for (int st = 0; st < kStages - 1; ++st) {
-    if (st < n) load_tile(st, st);
+    if (st < n) load_tile(st, fetch_slot(st));
     cp_async_commit();  // group st (group 0 also holds Q)
   }
+  long long slot_next = kStages - 1 < n ? fetch_slot(kStages - 1) : -1;  // tile j + kStages - 1
 
   const float scale = a.g.sm_scale_log2;
   const int r0 = lane >> 2;  // accumulator rows r0 and r0 + 8 (heads)
@@ -159,8 +165,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) mla_decode_kernel(const 
   for (int j = 0; j < n; ++j) {
     cp_async_wait<kStages - 2>();
     __syncthreads();  // tile j is in shared memory; every warp is done with tile j - 1
-    if (j + kStages - 1 < n) load_tile(j + kStages - 1, (j + kStages - 1) % kStages);
+    if (j + kStages - 1 < n) load_tile((j + kStages - 1) % kStages, slot_next);
     cp_async_commit();
+    if (j + kStages < n) slot_next = fetch_slot(j + kStages);
     const uint32_t cst = sbase + kOffStage + (j % kStages) * kStageBytes;
     const uint32_t kst = cst + kCkvBytes;
 
