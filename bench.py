@@ -238,6 +238,7 @@ class Case:
             self.q, self.k, self.v = p.q.to(device), p.k_cache.to(device), p.v_cache.to(device)
             if p.is_fp8_kv:
                 self.k_scale, self.v_scale = p.meta["k_scale"].to(device), p.meta["v_scale"].to(device)
+                plan_kw.setdefault("kv_fp8", True)
             self.plan = pkv.plan(p.qo_indptr, p.kv_indptr, self.idx, p.kv_last_page_len, p.num_qo_heads,
                                  p.num_kv_heads, p.head_dim, p.page_size, p.causal, p.sm_scale, **plan_kw)
             self.o = torch.empty(p.total_q, p.num_qo_heads, p.head_dim_v, dtype=torch.bfloat16, device=device)

@@ -97,7 +97,10 @@ typedef struct pkv_plan_options {
   int32_t kv_layout;        /* GQA/MHA page layout (FlashInfer 0.7.4 documentation, "KV-Cache Layout in
                                FlashInfer", "Layout: NHD/HND"): 0 = NHD, a page is [page_size, Hk, D];
                                1 = HND, a page is [Hk, page_size, D]. MLA pools have no head axis: ignored. */
-  int32_t reserved[4];
+  int32_t kv_fp8;           /* 1 = the plan is for pkv_run_fp8_kv: a decode plan's split-KV chunk is sized for
+                               that kernel's occupancy. Results do not depend on it; either run accepts either
+                               plan. Ignored by MLA and prefill plans. */
+  int32_t reserved[3];
 } pkv_plan_options;
 
 /* Plan a batch: builds the CTA work list on the host.

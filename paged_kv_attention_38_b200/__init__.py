@@ -42,7 +42,8 @@ class PkvError(RuntimeError):
 
 class _Options(ctypes.Structure):
     _fields_ = [("num_sms", ctypes.c_int32), ("disable_split_kv", ctypes.c_int32),
-                ("kv_chunk", ctypes.c_int32), ("kv_layout", ctypes.c_int32), ("reserved", ctypes.c_int32 * 4)]
+                ("kv_chunk", ctypes.c_int32), ("kv_layout", ctypes.c_int32), ("kv_fp8", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 3)]
 
 
 _lib = None
@@ -195,27 +196,30 @@ class Plan:
             _lib.pkv_plan_destroy(h)
 
 
-def _options(num_sms, disable_split_kv, kv_chunk, kv_layout=0):
+def _options(num_sms, disable_split_kv, kv_chunk, kv_layout=0, kv_fp8=False):
     o = _Options()
     o.num_sms, o.disable_split_kv, o.kv_chunk = int(num_sms), int(bool(disable_split_kv)), int(kv_chunk)
-    o.kv_layout = int(kv_layout)
+    o.kv_layout, o.kv_fp8 = int(kv_layout), int(bool(kv_fp8))
     return o
 
 
 def plan(qo_indptr, kv_indptr, kv_indices, kv_last_page_len, num_qo_heads, num_kv_heads, head_dim,
          page_size, causal, sm_scale, *, num_sms: int = 0, disable_split_kv: bool = False,
-         kv_chunk: int = 0, kv_layout: int = 0, upload: bool = True, device=None, stream=None) -> Plan:
+         kv_chunk: int = 0, kv_layout: int = 0, kv_fp8: bool = False, upload: bool = True, device=None,
+         stream=None) -> Plan:
     """Plan a GQA/MHA paged-attention batch (``pkv_plan_create`` + ``pkv_plan_upload``).
 
     ``qo_indptr``, ``kv_indptr``, ``kv_last_page_len`` are host int32 arrays;
     ``kv_indices`` is a device int32 tensor (may be None with ``upload=False``
     to inspect the schedule on a machine without a GPU). ``kv_layout``: 0 NHD
-    pools ``[num_pages, page_size, Hk, D]``, 1 HND ``[num_pages, Hk, page_size, D]``.
+    pools ``[num_pages, page_size, Hk, D]``, 1 HND ``[num_pages, Hk, page_size, D]``. ``kv_fp8``: the
+    plan will run through ``run_fp8_kv`` (its split-KV chunk is sized for that kernel; results do not
+    depend on it).
     """
     lib = load_library()
     qo, kv, last = _host_i32(qo_indptr), _host_i32(kv_indptr), _host_i32(kv_last_page_len)
     h = _P()
-    opts = _options(num_sms, disable_split_kv, kv_chunk, kv_layout)
+    opts = _options(num_sms, disable_split_kv, kv_chunk, kv_layout, kv_fp8)
     _check(lib.pkv_plan_create(_i32p(qo), _i32p(kv), _ptr(kv_indices), _i32p(last), len(last), num_qo_heads,
                                num_kv_heads, head_dim, page_size, int(bool(causal)), float(sm_scale),
                                ctypes.byref(opts), ctypes.byref(h)))

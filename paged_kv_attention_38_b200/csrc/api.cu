@@ -122,6 +122,7 @@ void fill_in(PlanInput& in, const int32_t* qo_indptr, const int32_t* kv_indptr, 
   in.disable_split_kv = opts ? opts->disable_split_kv : 0;
   in.kv_chunk = opts ? opts->kv_chunk : 0;
   in.kv_layout = opts ? opts->kv_layout : 0;
+  in.kv_fp8 = opts ? opts->kv_fp8 : 0;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }

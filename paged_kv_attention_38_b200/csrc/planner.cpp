@@ -39,6 +39,64 @@ struct Tile {
   int32_t req, kv_head, row0, rows, kv_need;
 };
 
+// GQA decode split model. A decode kernel is bound by HBM bandwidth, so what a
+// split buys is balance: the units (tile x KV chunk) are taken longest first by
+// `slots` resident CTAs, and the launch ends with its most loaded slot. Costs
+// are in keys: a unit costs its keys plus kDecodeUnitCost (prologue, Q load,
+// epilogue), and any split adds one merge launch, kDecodeMergeCost. Both
+// constants were fitted to measured launch times of decode batches on B200
+// (the model ranks chunk lengths as the measurements did; without the merge
+// cost it prefers splits that measured slower than none).
+constexpr int64_t kDecodeUnitCost = 256;
+constexpr int64_t kDecodeMergeCost = 400;
+
+// Makespan, in keys, of the units that chunk length `c` (0 = no split) cuts the
+// tiles into, when `slots` CTAs take them longest first. Full chunks all have
+// length c and are the longest units, so they are dealt round-robin; the
+// remainders (one per tile at most) go, longest first, to the least loaded
+// slot. `need` is sorted in descending order; `rem` and `heap` are scratch.
+int64_t decode_makespan(const std::vector<int64_t>& need, int64_t c, int64_t slots, std::vector<int64_t>& rem,
+                        std::vector<int64_t>& heap) {
+  int64_t full = 0;
+  rem.clear();
+  size_t whole = 0;  // need[whole..] fit one chunk and keep their sorted order
+  if (c > 0) {
+    while (whole < need.size() && need[whole] > c) {
+      full += need[whole] / c;
+      if (need[whole] % c) rem.push_back(need[whole] % c);
+      ++whole;
+    }
+    std::sort(rem.begin(), rem.end(), std::greater<int64_t>());
+  }
+  const int64_t k = full / slots, extra = full % slots;
+  heap.clear();
+  int64_t worst = 0;
+  for (int64_t i = 0; i < slots; ++i) {
+    const int64_t l = (k + (i < extra ? 1 : 0)) * (c + kDecodeUnitCost);
+    heap.push_back(l);
+    worst = std::max(worst, l);
+  }
+  std::make_heap(heap.begin(), heap.end(), std::greater<int64_t>());
+  auto place = [&](int64_t r) {
+    std::pop_heap(heap.begin(), heap.end(), std::greater<int64_t>());
+    heap.back() += r + kDecodeUnitCost;
+    worst = std::max(worst, heap.back());
+    std::push_heap(heap.begin(), heap.end(), std::greater<int64_t>());
+  };
+  // longest first: merge the sorted remainders with the sorted whole tiles
+  size_t i = 0, j = whole;
+  while (i < rem.size() || j < need.size()) {
+    if (j == need.size() || (i < rem.size() && rem[i] >= need[j])) place(rem[i++]);
+    else place(need[j++]);
+  }
+  return worst;
+}
+
+// Resident CTAs per SM of the GQA decode kernels on sm_100a (set by their
+// shared memory and registers): bf16 K/V 2 at head_dim 128, the FP8 kernel 3,
+// either 4 at head_dim 64.
+int64_t decode_ctas_per_sm(int32_t head_dim, bool fp8) { return head_dim <= 64 ? 4 : fp8 ? 3 : 2; }
+
 }  // namespace
 
 int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
@@ -147,9 +205,42 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   if (!in.disable_split_kv) {
     if (in.kv_chunk > 0) {
       chunk = round_up(in.kv_chunk, align);
-    } else if (s.kind == kKindDecode || s.kind == kKindMlaDecode) {
-      // Decode is HBM-bound: aim for ~8 units per SM so the tail is short; a
-      // chunk below 512 keys would spend more on partial state than it saves.
+    } else if (s.kind == kKindDecode) {
+      // Candidates from half the average load per slot up to the longest tile
+      // (x1.15 steps), and no split; the cheapest by decode_makespan wins.
+      // When no tile reaches half the average load, longest-first placement of
+      // whole tiles is already balanced: no split, and no search.
+      const int64_t slots = decode_ctas_per_sm(in.head_dim, in.kv_fp8 != 0) * (int64_t)num_sms;
+      std::vector<int64_t> need, rem, heap;
+      need.reserve(tiles.size());
+      int64_t total = 0;
+      for (const Tile& t : tiles) {
+        need.push_back(t.kv_need);
+        total += t.kv_need + kDecodeUnitCost;
+      }
+      std::sort(need.begin(), need.end(), std::greater<int64_t>());
+      const int64_t avg = total / std::max<int64_t>(1, slots);
+      if ((int64_t)max_need * 2 <= avg) {
+        chunk = 0;
+      } else if (tiles.size() > 8192) {
+        chunk = round_up(std::max<int64_t>(avg, 4 * align), align);  // too many tiles to search cheaply
+      } else {
+        int64_t best = 0, best_t = decode_makespan(need, 0, slots, rem, heap);
+        for (int64_t c = std::max<int64_t>(4 * align, round_up(avg / 2, align)); c < max_need;
+             c = std::max<int64_t>(c + align, (c * 115 / 100) / align * align)) {
+          const int64_t t_est = decode_makespan(need, c, slots, rem, heap) + kDecodeMergeCost;
+          if (t_est < best_t) {
+            best_t = t_est;
+            best = c;
+          }
+        }
+        chunk = best;
+      }
+    } else if (s.kind == kKindMlaDecode) {
+      // MLA decode is bound by each CTA's instruction chain rather than by HBM
+      // (few requests, all heads in one CTA): aim for ~8 units per SM so the
+      // tail is short; a chunk below 512 keys would spend more on partial state
+      // than it saves.
       chunk = round_up(std::max<int64_t>(512, total_cost / ((int64_t)num_sms * 8)), align);
       chunk = std::min<int64_t>(chunk, 4096);
       // Wave quantisation: units run two CTAs per SM in waves of 2 x SMs, and

@@ -33,6 +33,7 @@ struct PlanInput {
   int32_t disable_split_kv;
   int32_t kv_chunk;     // > 0 forces the split chunk
   int32_t kv_layout;    // 0 NHD, 1 HND (GQA/MHA pools)
+  int32_t kv_fp8;       // 1: a decode plan for the FP8-KV kernel (sizes its split for that kernel)
 };
 
 struct Schedule {

@@ -120,6 +120,31 @@ def test_planner_forced_split(chunk):
     assert pl.num_merges > 0
 
 
+@pytest.mark.parametrize("kv_fp8", [False, True])
+@pytest.mark.parametrize("kv", [[10000, 20000, 5, 7], [100000], [512] * 4, [1, 63, 64, 65, 700, 3000],
+                                [1024 + 61 * i for i in range(128)]])
+def test_planner_decode_split_choice(kv, kv_fp8):
+    """The decode split search: whatever chunk it picks is a multiple of the 64-key
+    tile, at least 256 keys, shorter than the longest request (else no split), and
+    the schedule covers every key exactly once."""
+    p = _lengths_problem([1] * len(kv), kv, hq=32, hk=8, d=128, ps=16, causal=False)
+    pl = _plan(p, kv_fp8=kv_fp8)
+    assert pl.kind == pkv.KIND_DECODE
+    c = pl.kv_chunk
+    assert c == 0 or (c % 64 == 0 and 256 <= c < max(kv)), c
+    assert (pl.num_merges > 0) == (c > 0 and max(kv) > c)
+    _check_coverage(p, pl)
+
+
+def test_planner_decode_split_balances_few_long_requests():
+    """Eight (request, kv head) tiles of 100k keys cannot fill 148 SMs: the plan
+    splits them into enough chunks for every SM."""
+    p = _lengths_problem([1], [100000], hq=32, hk=8, d=128, ps=16, causal=False)
+    pl = _plan(p)
+    assert pl.num_units >= 148 and pl.num_merges == 8
+    _check_coverage(p, pl)
+
+
 def test_planner_disable_split_kv():
     p = _lengths_problem([1] * 4, [10000, 20000, 5, 7], hq=8, hk=2, ps=16, causal=False)
     pl = _plan(p, disable_split_kv=True)

@@ -239,7 +239,8 @@ def test_decode_sweep(case, split):
 
 @pytest.mark.slow
 def test_decode_full_size():
-    """b128/h32/kv8/d128/ps16, kv_len 1024..8192, default split-KV plan: every row."""
+    """b128/h32/kv8/d128/ps16, kv_len 1024..8192, the planner's default plan (the bench's launch
+    configuration; it does not split this batch): every row."""
     p = W.paged_decode()
     o, lse, pl = gpu_run(p)
     assert pl.kind == pkv.KIND_DECODE
@@ -250,6 +251,7 @@ def test_decode_full_size():
 
 def gpu_run_fp8(p: W.PagedProblem, k_scale=True, v_scale=True, **plan_kw):
     d = to_dev(p)
+    plan_kw.setdefault("kv_fp8", True)
     pl = pkv.plan(p.qo_indptr, p.kv_indptr, d["kv_indices"], p.kv_last_page_len, p.num_qo_heads,
                   p.num_kv_heads, p.head_dim, p.page_size, p.causal, p.sm_scale, **plan_kw)
     ks = p.meta["k_scale"].cuda() if k_scale else None
