@@ -93,24 +93,27 @@ __device__ __forceinline__ void attend(uint8_t* smem, const Job& jb) {
   const int n = jb.kv_hi > jb.kv_lo ? (jb.kv_hi - jb.kv_lo + kTile - 1) / kTile : 0;
   const uint32_t sbase = smem_u32(smem);
 
+  // Each warp reads only its own 16 key rows of every stage (rows 16 warp +
+  // [0, 16)), so each warp also copies them itself and waits on its own copy
+  // groups: no CTA-wide barrier per tile, the warps run at their own pace.
   // All page-table reads of a tile are issued before its copies: a read inside
   // the copy loop would wait for the previous copy to be issued (the copies
   // are ordered memory operations), serialising one global read per copy.
-  constexpr int kPerThread = kTile * kChunks / kThreads;
-  static_assert(kTile * kChunks % kThreads == 0, "whole copies per thread");
+  constexpr int kPerLane = 16 * kChunks / 32;
+  static_assert(16 * kChunks % 32 == 0, "whole copies per lane");
   auto load_tile = [&](int j, int stage) {
     const uint32_t kdst = sbase + stage * 2 * kTileBytes;
     const uint32_t vdst = kdst + kTileBytes;
-    int page[kPerThread];
+    int page[kPerLane];
 #pragma unroll
-    for (int i = 0; i < kPerThread; ++i) {
-      const int pos = jb.kv_lo + j * kTile + (tid + i * kThreads) / kChunks;
+    for (int i = 0; i < kPerLane; ++i) {
+      const int pos = jb.kv_lo + j * kTile + warp * 16 + (lane + 32 * i) / kChunks;
       page[i] = pos < jb.kv_hi ? __ldg(jb.pages + (pos >> shift)) : -1;
     }
 #pragma unroll
-    for (int i = 0; i < kPerThread; ++i) {
-      const int c = tid + i * kThreads;
-      const int r = c / kChunks, ch = c % kChunks;
+    for (int i = 0; i < kPerLane; ++i) {
+      const int c = lane + 32 * i;
+      const int r = warp * 16 + c / kChunks, ch = c % kChunks;
       const int pos = jb.kv_lo + j * kTile + r;
       const bool ok = page[i] >= 0;
       size_t off = 0;
@@ -154,7 +157,7 @@ __device__ __forceinline__ void attend(uint8_t* smem, const Job& jb) {
 
   for (int j = 0; j < n; ++j) {
     cp_async_wait<kStages - 2>();
-    __syncthreads();
+    __syncwarp();  // this warp's rows of tile j have landed; its reads of tile j - 1 are done
     if (j + kStages - 1 < n) load_tile(j + kStages - 1, (j + kStages - 1) % kStages);
     cp_async_commit();
 

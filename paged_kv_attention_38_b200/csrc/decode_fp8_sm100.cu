@@ -122,14 +122,17 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
   const int n = (unit.kv_hi - unit.kv_lo + kTile - 1) / kTile;
   const uint32_t sbase = smem_u32(smem);
 
+  // Each warp reads only its own 16 key rows of every stage (rows 16 warp +
+  // [0, 16)), so each warp also copies them itself and waits on its own copy
+  // groups: no CTA-wide barrier per tile, the warps run at their own pace.
   // Page ids are read one tile ahead of the copies that use them, during the
   // previous tile's math, so no warp waits a global-memory latency per tile.
-  constexpr int kPerThread = kTile * kChunks / kThreads;
-  static_assert(kTile * kChunks % kThreads == 0, "whole copies per thread");
+  constexpr int kPerLane = 16 * kChunks / 32;
+  static_assert(16 * kChunks % 32 == 0, "whole copies per lane");
   auto fetch_pages = [&](int j, int* page) {
 #pragma unroll
-    for (int i = 0; i < kPerThread; ++i) {
-      const int pos = unit.kv_lo + j * kTile + (tid + i * kThreads) / kChunks;
+    for (int i = 0; i < kPerLane; ++i) {
+      const int pos = unit.kv_lo + j * kTile + warp * 16 + (lane + 32 * i) / kChunks;
       page[i] = pos < unit.kv_hi ? __ldg(a.kv_indices + req.page0 + (pos >> shift)) : -1;
     }
   };
@@ -137,9 +140,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
     const uint32_t kdst = sbase + stage * 2 * kCodeTile;
     const uint32_t vdst = kdst + kCodeTile;
 #pragma unroll
-    for (int i = 0; i < kPerThread; ++i) {
-      const int c = tid + i * kThreads;
-      const int r = c / kChunks, ch = c % kChunks;
+    for (int i = 0; i < kPerLane; ++i) {
+      const int c = lane + 32 * i;
+      const int r = warp * 16 + c / kChunks, ch = c % kChunks;
       const int pos = unit.kv_lo + j * kTile + r;
       const bool ok = page[i] >= 0;
       const size_t off = ok ? (((size_t)page[i] * P + (pos & (P - 1))) * Hk + unit.kv_head) * D + ch * 16 : 0;
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
     }
   };
 
-  int page_next[kPerThread];  // ids of tile (j + kStages - 1), read during tile j - 1
+  int page_next[kPerLane];  // ids of tile (j + kStages - 1), read during tile j - 1
 #pragma unroll
   for (int s = 0; s < kStages - 1; ++s) {
     if (s < n) {
@@ -211,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
 
   for (int j = 0; j < n; ++j) {
     cp_async_wait<kStages - 2>();
-    __syncthreads();
+    __syncwarp();  // this warp's rows of tile j have landed; its reads of tile j - 1 are done
     if (j + kStages - 1 < n) load_tile(j + kStages - 1, (j + kStages - 1) % kStages, page_next);
     cp_async_commit();
     if (j + kStages < n) fetch_pages(j + kStages, page_next);

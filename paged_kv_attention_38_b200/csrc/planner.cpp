@@ -39,9 +39,9 @@ struct Tile {
   int32_t req, kv_head, row0, rows, kv_need;
 };
 
-// GQA decode split model. A decode kernel is bound by HBM bandwidth, so what a
-// split buys is balance: the units (tile x KV chunk) are taken longest first by
-// `slots` resident CTAs, and the launch ends with its most loaded slot. Costs
+// Decode split model (GQA and MLA decode). What a split buys is balance: the
+// units (tile x KV chunk) are taken longest first by `slots` resident CTAs,
+// and the launch ends with its most loaded slot. Costs
 // are in keys: a unit costs its keys plus kDecodeUnitCost (prologue, Q load,
 // epilogue), and any split adds one merge launch, kDecodeMergeCost. Both
 // constants were fitted to measured launch times of decode batches on B200
@@ -92,10 +92,13 @@ int64_t decode_makespan(const std::vector<int64_t>& need, int64_t c, int64_t slo
   return worst;
 }
 
-// Resident CTAs per SM of the GQA decode kernels on sm_100a (set by their
-// shared memory and registers): bf16 K/V 2 at head_dim 128, the FP8 kernel 3,
-// either 4 at head_dim 64.
-int64_t decode_ctas_per_sm(int32_t head_dim, bool fp8) { return head_dim <= 64 ? 4 : fp8 ? 3 : 2; }
+// Resident CTAs per SM of the decode kernels on sm_100a (set by their shared
+// memory and registers): GQA with bf16 K/V 2 at head_dim 128, the FP8 kernel 3,
+// either 4 at head_dim 64; MLA decode 2.
+int64_t decode_ctas_per_sm(KernelKind kind, int32_t head_dim, bool fp8) {
+  if (kind == kKindMlaDecode) return 2;
+  return head_dim <= 64 ? 4 : fp8 ? 3 : 2;
+}
 
 }  // namespace
 
@@ -205,12 +208,12 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
   if (!in.disable_split_kv) {
     if (in.kv_chunk > 0) {
       chunk = round_up(in.kv_chunk, align);
-    } else if (s.kind == kKindDecode) {
+    } else if (s.kind == kKindDecode || s.kind == kKindMlaDecode) {
       // Candidates from half the average load per slot up to the longest tile
       // (x1.15 steps), and no split; the cheapest by decode_makespan wins.
       // When no tile reaches half the average load, longest-first placement of
       // whole tiles is already balanced: no split, and no search.
-      const int64_t slots = decode_ctas_per_sm(in.head_dim, in.kv_fp8 != 0) * (int64_t)num_sms;
+      const int64_t slots = decode_ctas_per_sm(s.kind, in.head_dim, in.kv_fp8 != 0) * (int64_t)num_sms;
       std::vector<int64_t> need, rem, heap;
       need.reserve(tiles.size());
       int64_t total = 0;
@@ -236,29 +239,6 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
         }
         chunk = best;
       }
-    } else if (s.kind == kKindMlaDecode) {
-      // MLA decode is bound by each CTA's instruction chain rather than by HBM
-      // (few requests, all heads in one CTA): aim for ~8 units per SM so the
-      // tail is short; a chunk below 512 keys would spend more on partial state
-      // than it saves.
-      chunk = round_up(std::max<int64_t>(512, total_cost / ((int64_t)num_sms * 8)), align);
-      chunk = std::min<int64_t>(chunk, 4096);
-      // Wave quantisation: units run two CTAs per SM in waves of 2 x SMs, and
-      // a last wave that is nearly empty costs as much as a full one. Among
-      // chunks up to 2x the first guess take the one with the smallest
-      // (waves x chunk), the time model of equal, full-chunk units.
-      const int64_t wave = 2 * (int64_t)num_sms;
-      int64_t best = chunk, best_t = INT64_MAX;
-      for (int64_t c = chunk; c <= 2 * chunk; c += align) {
-        int64_t units = 0;
-        for (const Tile& t : tiles) units += (t.kv_need + c - 1) / c;
-        const int64_t t_est = (units + wave - 1) / wave * std::min<int64_t>(c, max_need);
-        if (t_est < best_t) {
-          best_t = t_est;
-          best = c;
-        }
-      }
-      chunk = best;
     } else {
       // Prefill: one CTA per SM at a time; split only when a single tile is
       // longer than the average work per SM.
