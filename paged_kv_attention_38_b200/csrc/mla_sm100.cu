@@ -406,33 +406,70 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
       const float lse2 = l_row > 0.f ? m_row + __log2f(l_row) : -INFINITY;
       const int half = s_owner ? 0 : 1;
       const size_t orow = (size_t)(req.q_start + t) * H + pr % H;
-      for (int c = 0; c < 256; c += 32) {
-        float ov[32];
-        if (n_tiles > 0) {
-          tmem_ld32(lane_base + c, ov);
-          tmem_ld_wait();
-        } else {
+      if (unit.partial >= 0) {
+        for (int c = 0; c < 256; c += 32) {
+          float ov[32];
+          if (n_tiles > 0) {
+            tmem_ld32(lane_base + c, ov);
+            tmem_ld_wait();
+          } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) ov[x] = 0.f;
-        }
-        if (!row_ok) continue;
-        const int d0 = half * 256 + c;
-        if (unit.partial >= 0) {
-          float* dst = a.dv.part_o + ((size_t)unit.partial * kRows + row) * kDc + d0;
+            for (int x = 0; x < 32; ++x) ov[x] = 0.f;
+          }
+          if (!row_ok) continue;
+          float* dst = a.dv.part_o + ((size_t)unit.partial * kRows + row) * kDc + half * 256 + c;
 #pragma unroll
           for (int x = 0; x < 32; x += 4)
             *reinterpret_cast<float4*>(dst + x) =
                 make_float4(ov[x] * inv_l, ov[x + 1] * inv_l, ov[x + 2] * inv_l, ov[x + 3] * inv_l);
-        } else {
-          __nv_bfloat16* dst = a.o + orow * kDc + d0;
+        }
+      } else {
+        // bf16 O, 64 columns of the thread's half-row at a time: 8 pieces of
+        // 16 bytes. Each group of 8 lanes transposes its 8 half-rows x 8
+        // pieces with xor butterflies, so that one store instruction writes
+        // four whole 128-byte lines (lane 8g + i: piece i of half-row 8g + k)
+        // instead of 32 pieces of 32 different lines.
+        const int grp = lane & ~7, li = lane & 7;
+        const size_t orow0 = (size_t)req.q_start * H + unit.row0;
+        for (int c = 0; c < 256; c += 64) {
+          float ov[64];
+          if (n_tiles > 0) {
+            tmem_ld32(lane_base + c, ov);
+            tmem_ld32(lane_base + c + 32, ov + 32);
+            tmem_ld_wait();
+          } else {
 #pragma unroll
-          for (int x = 0; x < 32; x += 8) {
-            uint4 w;
-            w.x = pack_bf16x2(ov[x + 0] * inv_l, ov[x + 1] * inv_l);
-            w.y = pack_bf16x2(ov[x + 2] * inv_l, ov[x + 3] * inv_l);
-            w.z = pack_bf16x2(ov[x + 4] * inv_l, ov[x + 5] * inv_l);
-            w.w = pack_bf16x2(ov[x + 6] * inv_l, ov[x + 7] * inv_l);
-            *reinterpret_cast<uint4*>(dst + x) = w;
+            for (int x = 0; x < 64; ++x) ov[x] = 0.f;
+          }
+          uint4 pc[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            pc[k] = make_uint4(pack_bf16x2(ov[8 * k + 0] * inv_l, ov[8 * k + 1] * inv_l),
+                               pack_bf16x2(ov[8 * k + 2] * inv_l, ov[8 * k + 3] * inv_l),
+                               pack_bf16x2(ov[8 * k + 4] * inv_l, ov[8 * k + 5] * inv_l),
+                               pack_bf16x2(ov[8 * k + 6] * inv_l, ov[8 * k + 7] * inv_l));
+#pragma unroll
+          for (int sbit = 1; sbit < 8; sbit <<= 1) {
+            const bool upper = (li & sbit) != 0;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              if (k & sbit) continue;
+              uint4 snd = upper ? pc[k] : pc[k ^ sbit];
+              uint4 rcv;
+              rcv.x = __shfl_xor_sync(0xffffffffu, snd.x, sbit);
+              rcv.y = __shfl_xor_sync(0xffffffffu, snd.y, sbit);
+              rcv.z = __shfl_xor_sync(0xffffffffu, snd.z, sbit);
+              rcv.w = __shfl_xor_sync(0xffffffffu, snd.w, sbit);
+              if (upper) pc[k] = rcv;
+              else pc[k ^ sbit] = rcv;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int src = grp + k;               // lane whose half-row this store writes
+            const int r = warp * 16 + (src & 15);  // its row of the unit
+            if (r < unit.rows)
+              *reinterpret_cast<uint4*>(a.o + (orow0 + r) * kDc + (src >> 4) * 256 + c + 8 * li) = pc[k];
           }
         }
       }
