@@ -608,27 +608,52 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
           }
           if (row_ok) a.dv.part_lse[(size_t)unit.partial * kPrefillUnitRows + ru] = lse2;
         } else {
-          __nv_bfloat16* dst = a.o + ((size_t)tok * a.g.num_qo_heads + h) * D;
+          // 64 columns of the row at a time (8 pieces of 16 bytes). Each group
+          // of 8 lanes (8 consecutive rows) transposes its 8 rows x 8 pieces
+          // with xor butterflies, so that one store instruction writes four
+          // 128-byte runs (lane 8g + i: piece i of row 8g + k) instead of 32
+          // pieces of 32 different lines. A row's address comes from its lane.
+          char* my_dst = row_ok ? reinterpret_cast<char*>(a.o + ((size_t)tok * a.g.num_qo_heads + h) * D) : nullptr;
+          const int li = lane & 7, grp = lane & ~7;
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            float ov[32];
+          for (int c = 0; c < D; c += 64) {
+            float ov[64];
             if (n_tiles > 0) {
               tmem_ld32(o_tm + c, ov);
+              tmem_ld32(o_tm + c + 32, ov + 32);
               tmem_ld_wait();
             } else {
 #pragma unroll
-              for (int x = 0; x < 32; ++x) ov[x] = 0.f;
+              for (int x = 0; x < 64; ++x) ov[x] = 0.f;
             }
-            if (row_ok) {
+            uint4 pc[8];
 #pragma unroll
-              for (int x = 0; x < 32; x += 8) {
-                uint4 w;
-                w.x = pack_bf16x2(ov[x + 0] * inv_l, ov[x + 1] * inv_l);
-                w.y = pack_bf16x2(ov[x + 2] * inv_l, ov[x + 3] * inv_l);
-                w.z = pack_bf16x2(ov[x + 4] * inv_l, ov[x + 5] * inv_l);
-                w.w = pack_bf16x2(ov[x + 6] * inv_l, ov[x + 7] * inv_l);
-                *reinterpret_cast<uint4*>(dst + c + x) = w;
+            for (int k = 0; k < 8; ++k)
+              pc[k] = make_uint4(pack_bf16x2(ov[8 * k + 0] * inv_l, ov[8 * k + 1] * inv_l),
+                                 pack_bf16x2(ov[8 * k + 2] * inv_l, ov[8 * k + 3] * inv_l),
+                                 pack_bf16x2(ov[8 * k + 4] * inv_l, ov[8 * k + 5] * inv_l),
+                                 pack_bf16x2(ov[8 * k + 6] * inv_l, ov[8 * k + 7] * inv_l));
+#pragma unroll
+            for (int sbit = 1; sbit < 8; sbit <<= 1) {
+              const bool upper = (li & sbit) != 0;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                if (k & sbit) continue;
+                const uint4 snd = upper ? pc[k] : pc[k ^ sbit];
+                uint4 rcv;
+                rcv.x = __shfl_xor_sync(0xffffffffu, snd.x, sbit);
+                rcv.y = __shfl_xor_sync(0xffffffffu, snd.y, sbit);
+                rcv.z = __shfl_xor_sync(0xffffffffu, snd.z, sbit);
+                rcv.w = __shfl_xor_sync(0xffffffffu, snd.w, sbit);
+                if (upper) pc[k] = rcv;
+                else pc[k ^ sbit] = rcv;
               }
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              char* d = reinterpret_cast<char*>(
+                  __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), grp + k));
+              if (d) *reinterpret_cast<uint4*>(d + c * 2 + li * 16) = pc[k];
             }
           }
           if (row_ok && a.lse) a.lse[(size_t)tok * a.g.num_qo_heads + h] = lse2;
