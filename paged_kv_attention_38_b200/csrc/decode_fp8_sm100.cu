@@ -129,7 +129,15 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
   // previous tile's math, so no warp waits a global-memory latency per tile.
   constexpr int kPerLane = 16 * kChunks / 32;
   static_assert(16 * kChunks % 32 == 0, "whole copies per lane");
+  // With pages of 16 keys or more, a warp's 16 rows (16-aligned positions) lie
+  // in one page: one page id per lane, and the rows' offsets step by Hk * D.
+  const bool one_page = P >= 16;
   auto fetch_pages = [&](int j, int* page) {
+    if (one_page) {
+      const int pos = unit.kv_lo + j * kTile + warp * 16;
+      page[0] = pos < unit.kv_hi ? __ldg(a.kv_indices + req.page0 + (pos >> shift)) : -1;
+      return;
+    }
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
       const int pos = unit.kv_lo + j * kTile + warp * 16 + (lane + 32 * i) / kChunks;
@@ -139,6 +147,21 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
   auto load_tile = [&](int j, int stage, const int* page) {
     const uint32_t kdst = sbase + stage * 2 * kCodeTile;
     const uint32_t vdst = kdst + kCodeTile;
+    if (one_page) {
+      const int pos0 = unit.kv_lo + j * kTile + warp * 16;
+      const size_t base =
+          page[0] >= 0 ? (((size_t)page[0] * P + (pos0 & (P - 1))) * Hk + unit.kv_head) * D : 0;
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i) {
+        const int c = lane + 32 * i;
+        const int rr = c / kChunks, ch = c % kChunks;
+        const bool ok = page[0] >= 0 && pos0 + rr < unit.kv_hi;
+        const size_t off = ok ? base + (size_t)rr * Hk * D + ch * 16 : 0;
+        cp_async_16(kdst + code_off<D>(warp * 16 + rr, ch), a.k + off, ok ? 16u : 0u);
+        cp_async_16(vdst + code_off<D>(warp * 16 + rr, ch), a.v + off, ok ? 16u : 0u);
+      }
+      return;
+    }
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
       const int c = lane + 32 * i;
@@ -243,13 +266,20 @@ __global__ void __launch_bounds__(kThreads, 3) decode_fp8_kernel(const __grid_co
       }
     }
     // mask keys past the unit's end, scale into the base-2 domain
-    const int key0 = unit.kv_lo + j * kTile + r0 + lc * 2;
+    if (unit.kv_lo + (j + 1) * kTile <= unit.kv_hi) {  // the whole tile is in range (warp-uniform)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = key0 + nt * 8 + (e & 1);
-        s[nt][e] = key < unit.kv_hi ? s[nt][e] * scale : -INFINITY;
+        for (int e = 0; e < 4; ++e) s[nt][e] *= scale;
+    } else {
+      const int key0 = unit.kv_lo + j * kTile + r0 + lc * 2;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = key0 + nt * 8 + (e & 1);
+          s[nt][e] = key < unit.kv_hi ? s[nt][e] * scale : -INFINITY;
+        }
       }
     }
     float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
