@@ -101,9 +101,29 @@ __device__ __forceinline__ void attend(uint8_t* smem, const Job& jb) {
   // are ordered memory operations), serialising one global read per copy.
   constexpr int kPerLane = 16 * kChunks / 32;
   static_assert(16 * kChunks % 32 == 0, "whole copies per lane");
+  // With pages of 16 keys or more, a warp's 16 rows (16-aligned positions) lie
+  // in one page: one page id per lane, and the rows' offsets step by a constant.
   auto load_tile = [&](int j, int stage) {
     const uint32_t kdst = sbase + stage * 2 * kTileBytes;
     const uint32_t vdst = kdst + kTileBytes;
+    if (P >= 16) {
+      const int pos0 = jb.kv_lo + j * kTile + warp * 16;
+      const int pg = pos0 < jb.kv_hi ? __ldg(jb.pages + (pos0 >> shift)) : -1;
+      const size_t base = pg < 0 ? 0
+                          : kHnd ? (((size_t)pg * Hk + jb.kv_head) * P + (pos0 & (P - 1))) * D
+                                 : (((size_t)pg * P + (pos0 & (P - 1))) * Hk + jb.kv_head) * D;
+      const size_t row_step = kHnd ? (size_t)D : (size_t)Hk * D;
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i) {
+        const int c = lane + 32 * i;
+        const int rr = c / kChunks, ch = c % kChunks;
+        const bool ok = pg >= 0 && pos0 + rr < jb.kv_hi;
+        const size_t off = ok ? base + rr * row_step + ch * 8 : 0;
+        cp_async_16(kdst + kv_off<D>(warp * 16 + rr, ch), jb.k + off, ok ? 16u : 0u);
+        cp_async_16(vdst + kv_off<D>(warp * 16 + rr, ch), jb.v + off, ok ? 16u : 0u);
+      }
+      return;
+    }
     int page[kPerLane];
 #pragma unroll
     for (int i = 0; i < kPerLane; ++i) {
@@ -177,13 +197,20 @@ __device__ __forceinline__ void attend(uint8_t* smem, const Job& jb) {
       }
     }
     // mask keys past the range's end, scale into the base-2 domain
-    const int key0 = jb.kv_lo + j * kTile + warp * 16 + (lane & 3) * 2;
+    if (jb.kv_lo + (j + 1) * kTile <= jb.kv_hi) {  // the whole tile is in range (warp-uniform)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = key0 + nt * 8 + (e & 1);
-        s[nt][e] = key < jb.kv_hi ? s[nt][e] * scale : -INFINITY;
+        for (int e = 0; e < 4; ++e) s[nt][e] *= scale;
+    } else {
+      const int key0 = jb.kv_lo + j * kTile + warp * 16 + (lane & 3) * 2;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = key0 + nt * 8 + (e & 1);
+          s[nt][e] = key < jb.kv_hi ? s[nt][e] * scale : -INFINITY;
+        }
       }
     }
     float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
