@@ -48,15 +48,23 @@ namespace {
 constexpr int kTileM = 128;
 constexpr int kTiles = 2;
 constexpr int kSlots = 4;
-constexpr int kThreads = 384;
+// Threads per CTA: 8 softmax warps, the MMA warp and the producer warps, 3 of
+// them for the page-TMA instance (one lane issues TMA), 7 for the row-gather
+// instance (its copy rate grows with the warps that issue 16-byte copies).
+template <bool kRows>
+constexpr int kThreadsOf = kRows ? 512 : 384;
 constexpr int kMmaWarp = 8;
 constexpr int kProdWarp0 = 9;
-constexpr int kProdThreads = 96;
+template <bool kRows>
+constexpr int kProdThreadsOf = kThreadsOf<kRows> - kProdWarp0 * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
-constexpr int kRegsSupport = 96;
+template <bool kRows>
+constexpr int kRegsSupportOf = kRows ? 56 : 96;
 constexpr int kRegsSoftmax = 200;
-static_assert(128 * kRegsSupport + 256 * kRegsSoftmax <= kThreads * 168, "register split exceeds the launch budget");
+// registers at launch: 65536 / threads, rounded down to a multiple of 8
+static_assert(128 * kRegsSupportOf<false> + 256 * kRegsSoftmax <= 384 * 168, "register split exceeds the launch budget");
+static_assert(256 * kRegsSupportOf<true> + 256 * kRegsSoftmax <= 512 * 128, "register split exceeds the launch budget");
 static_assert(kTileM * kTiles == kPrefillUnitRows, "unit rows");
 
 // Byte offset of 16-byte chunk `ch` of row `r` in a [128 x D] bf16 tile held as
@@ -113,7 +121,9 @@ struct Args {
 // tensor core starts its first QK^T while the softmax warps still write the
 // previous unit's output.
 template <int D, bool kRows, bool kHnd>
-__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Args a) {
+__global__ void __launch_bounds__(kThreadsOf<kRows>, 1) prefill_kernel(const __grid_constant__ Args a) {
+  constexpr int kProdThreads = kProdThreadsOf<kRows>;
+  constexpr int kRegsSupport = kRegsSupportOf<kRows>;
   extern __shared__ uint8_t smem_raw[];
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
@@ -150,10 +160,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   WaitCtx wc{&sm.abort_flag, a.dv.status};
-  // Registers: 384 threads x 168 at launch = 64512. The MMA/producer warpgroup
-  // (warps 8-11) drops to kRegsSupport, the two softmax warpgroups rise to
-  // kRegsSoftmax: 128 x 96 + 256 x 200 = 63488 <= 64512. Each role's code sits under its own
-  // setmaxnreg so the compiler allocates it with that budget.
+  // Registers: 384 threads x 168 at launch = 64512 (page instance) or 512 x 128
+  // = 65536 (row gather). The MMA/producer warpgroups (warps 8 and up) drop to
+  // kRegsSupport, the two softmax warpgroups rise to kRegsSoftmax: 128 x 96 +
+  // 256 x 200 = 63488 <= 64512, 256 x 56 + 256 x 200 = 65536. Each role's code
+  // sits under its own setmaxnreg so the compiler allocates it with that budget.
   if (warp >= kMmaWarp) {
     setmaxnreg_dec<kRegsSupport>();
   if (warp >= kProdWarp0) {
@@ -691,7 +702,7 @@ cudaError_t launch_as(const Args& a, cudaStream_t stream) {
   static std::atomic<uint64_t> configured{0};
   cudaError_t e = set_smem_attrs_once((const void*)prefill_kernel<D, kRows, kHnd>, (int)smem, configured, false);
   if (e != cudaSuccess) return e;
-  prefill_kernel<D, kRows, kHnd><<<a.g.num_ctas, kThreads, smem, stream>>>(a);
+  prefill_kernel<D, kRows, kHnd><<<a.g.num_ctas, kThreadsOf<kRows>, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
