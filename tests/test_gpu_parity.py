@@ -108,6 +108,8 @@ WIDE = [
     ([300, 129], [300, 129], 16, 4, 128, 256, True, 0),     # page_size 256: two KV tiles per page
     ([90, 250], [700, 250], 8, 2, 64, 256, True, 128),      # page_size 256, chunks starting mid-page
     ([160], [160], 12, 4, 128, 128, False, 0),              # group 3 with page_size 128, non-causal
+    ([200, 45], [200, 45], 24, 8, 128, 1, True, 0),         # group 3, page_size 1: cp.async Q + row gather
+    ([120, 300], [220, 300], 20, 4, 64, 2, True, 128),      # group 5, page_size 2, chunked, split KV (fp32 partials)
 ]
 
 
@@ -588,6 +590,7 @@ HND = [
     ([1, 1, 1], [70, 300, 5], 8, 2, 128, 16, False),  # decode kernel
     ([70, 300], [70, 300], 8, 2, 128, 128, True),   # page_size 128: one kv head's 128 slots per box
     ([1, 1], [600, 90], 24, 8, 64, 256, False),     # decode, group 3, page_size 256
+    ([100, 64], [100, 64], 12, 4, 128, 4, True),    # row gather with group 3 (cp.async Q)
 ]
 
 
