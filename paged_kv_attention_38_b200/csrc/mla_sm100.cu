@@ -54,7 +54,7 @@ namespace pkv {
 namespace {
 
 constexpr int kRows = kMlaUnitRows;  // 64
-constexpr int kN = 32;               // keys per latent tile
+constexpr int kN = kMlaTileN;        // keys per latent tile (32)
 constexpr int kStages = 4;
 constexpr int kDc = 512;
 constexpr int kDr = 64;

@@ -10,6 +10,7 @@ namespace pkv {
 constexpr int kBlockM = 128;   // packed (token, head-in-group) rows per tensor-core tile (TMEM lanes)
 constexpr int kPrefillUnitRows = 256;  // packed rows per prefill work unit (two tiles share K/V)
 constexpr int kMlaUnitRows = 64;       // packed (token, head) rows per MLA work unit (M = 64 MMAs)
+constexpr int kMlaTileN = 32;          // latent keys per MLA prefill tile
 constexpr int kBlockN = 128;   // KV slots per prefill KV tile
 constexpr int kDecodeRows = 16;  // packed rows per decode unit (mma.sync M)
 constexpr int kDecodeTileN = 64;  // KV slots per decode pipeline stage

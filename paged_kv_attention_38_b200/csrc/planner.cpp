@@ -304,12 +304,16 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
 
   // Prefill and MLA prefill run persistent CTAs (one per SM), each over a
   // fixed list of units. Greedy list scheduling in the longest-first order
-  // above: each unit goes to the CTA with the least work so far, counted in KV
-  // tiles plus one tile for the unit's own start and end. The units are then
-  // stored CTA by CTA.
+  // above: each unit goes to the CTA with the least work so far, counted in
+  // keys of whole KV tiles of the kernel plus the unit's own start and end:
+  // one 128-key tile for the prefill, two and a half 32-key tiles for the MLA
+  // prefill, whose unit boundary (the next unit's Q load and this unit's
+  // output) measured that long in a clock64 trace. The units are then stored
+  // CTA by CTA.
   int32_t num_ctas = (int32_t)s.units.size();
   if ((s.kind == kKindPrefill || s.kind == kKindMla) && !s.units.empty()) {
-    const int32_t tile = s.kind == kKindMla ? 64 : kBlockN;
+    const int64_t tile = s.kind == kKindMla ? kMlaTileN : kBlockN;
+    const int64_t edge = s.kind == kKindMla ? 5 * kMlaTileN / 2 : kBlockN;
     num_ctas = (int32_t)std::min<size_t>((size_t)num_sms, s.units.size());
     using Load = std::pair<int64_t, int32_t>;  // (work so far, cta)
     std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
@@ -319,7 +323,7 @@ int build_schedule(const PlanInput& in, Schedule* out, std::string* err) {
       Load top = heap.top();
       heap.pop();
       lists[(size_t)top.second].push_back(u);
-      top.first += (u.kv_hi - u.kv_lo + tile - 1) / tile + 1;
+      top.first += (u.kv_hi - u.kv_lo + tile - 1) / tile * tile + edge;
       heap.push(top);
     }
     s.units.clear();
