@@ -97,9 +97,11 @@ typedef struct pkv_plan_options {
   int32_t kv_layout;        /* GQA/MHA page layout (FlashInfer 0.7.4 documentation, "KV-Cache Layout in
                                FlashInfer", "Layout: NHD/HND"): 0 = NHD, a page is [page_size, Hk, D];
                                1 = HND, a page is [Hk, page_size, D]. MLA pools have no head axis: ignored. */
-  int32_t kv_fp8;           /* 1 = the plan is for pkv_run_fp8_kv: a decode plan's split-KV chunk is sized for
-                               that kernel's occupancy. Results do not depend on it; either run accepts either
-                               plan. Ignored by MLA and prefill plans. */
+  int32_t kv_fp8;           /* 1 = the plan is for pkv_run_fp8_kv. A decode plan's split-KV chunk is then sized
+                               for the FP8 kernel's occupancy (results do not depend on it; either run accepts
+                               either decode plan). A prefill plan reserves workspace for a bf16 copy of the
+                               batch's pages, which pkv_run_fp8_kv needs (about 4 bytes per page element more).
+                               Ignored by MLA plans. */
   int32_t reserved[3];
 } pkv_plan_options;
 
@@ -149,7 +151,7 @@ PKV_API pkv_status pkv_run(const pkv_plan* plan, const void* q, const void* k_ca
 PKV_API pkv_status pkv_run_mla(const pkv_plan* plan, const void* q_nope, const void* q_pe, const void* ckv_cache,
                        const void* kpe_cache, int32_t num_pages, void* o, float* lse, void* stream);
 
-/* Paged decode over a per-head-scale quantised KV cache ("[Roadmap]
+/* Paged attention over a per-head-scale quantised KV cache ("[Roadmap]
  * FlashInfer v0.2 to v0.3", milestone "Per Head Scale Quantized KV-Cache").
  * The pools hold FP8 E4M3 codes (OCP 8-bit floating point: 1 sign bit, 4
  * exponent bits with bias 7, 3 mantissa bits, exponent field 0 subnormal,
@@ -157,16 +159,24 @@ PKV_API pkv_status pkv_run_mla(const pkv_plan* plan, const void* q_nope, const v
  *   k_codes, v_codes  uint8 [num_pages, page_size, num_kv_heads, head_dim]  DEVICE
  *   k_scale, v_scale  fp32  [num_kv_heads]  DEVICE, or NULL for 1.0
  * The cache's value is decode(code) * scale[kv head], and the result is
- * pkv_run's attention over those values: q, o, lse as there. The plan must be
- * a decode plan from pkv_plan_create (every qo_len <= 1, group <= 16) with the
- * NHD layout and head_dim 64 or 128; anything else returns PKV_EUNSUPPORTED.
- * On the device each CTA scales its Q rows by a power of two that brings their
- * largest |q| to [2^13, 2^14) (undone exactly in the score scale) and rounds
- * them to f16, so any finite bf16 q is accepted; P is rounded to f16, every
- * code converts exactly to f16, and O and the LSE accumulate in fp32; NaN
- * codes propagate. Pointers 16-byte aligned; num_pages as in
- * pkv_run. Never allocates, never synchronises; the split-KV merge runs on the
- * same stream. */
+ * pkv_run's attention over those values: q, o, lse as there. The plan is a
+ * pkv_plan_create plan with the NHD layout and head_dim 64 or 128 (anything
+ * else returns PKV_EUNSUPPORTED), either
+ *   - a decode plan (every qo_len <= 1, group <= 16): one kernel reads the
+ *     codes directly. On the device each CTA scales its Q rows by a power of
+ *     two that brings their largest |q| to [2^13, 2^14) (undone exactly in the
+ *     score scale) and rounds them to f16, so any finite bf16 q is accepted; P
+ *     is rounded to f16, every code converts exactly to f16, and O and the LSE
+ *     accumulate in fp32; or
+ *   - a prefill plan made with pkv_plan_options.kv_fp8 = 1 (else
+ *     PKV_EUNSUPPORTED): a first kernel writes the batch's pages as bf16 (every
+ *     E4M3 value is exact in bf16; slots past a request's last key as zeros)
+ *     into the plan's workspace, and the tensor-core prefill of pkv_run runs
+ *     on that copy with K's scale applied to the scores and V's to the output;
+ *     Q and P are bf16 as in pkv_run. The scales must then be positive.
+ * NaN codes in a request's keys propagate. Pointers 16-byte aligned; num_pages
+ * as in pkv_run. Never allocates, never synchronises; the split-KV merge runs
+ * on the same stream. */
 PKV_API pkv_status pkv_run_fp8_kv(const pkv_plan* plan, const void* q, const void* k_codes, const void* v_codes,
                                   const float* k_scale, const float* v_scale, int32_t num_pages, void* o,
                                   float* lse, void* stream);

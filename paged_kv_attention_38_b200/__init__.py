@@ -293,9 +293,10 @@ def run_mla(p: Plan, q_nope, q_pe, ckv_cache, kpe_cache, o=None, lse=None, strea
 
 
 def run_fp8_kv(p: Plan, q, k_codes, v_codes, k_scale=None, v_scale=None, o=None, lse=None, stream=None):
-    """``pkv_run_fp8_kv``: decode over FP8 E4M3 K/V pools (``torch.float8_e4m3fn``
+    """``pkv_run_fp8_kv``: attention over FP8 E4M3 K/V pools (``torch.float8_e4m3fn``
     or ``uint8`` codes, NHD) with optional per-kv-head fp32 scales
-    ``[num_kv_heads]``. Returns ``(o bf16 [total_q, Hq, D], lse fp32 [total_q, Hq])``."""
+    ``[num_kv_heads]``, for a decode plan or a prefill plan made with
+    ``kv_fp8=True``. Returns ``(o bf16 [total_q, Hq, D], lse fp32 [total_q, Hq])``."""
     import torch
     _check_tensor(q, "q", torch.bfloat16)
     for t, n in ((k_codes, "k_codes"), (v_codes, "v_codes")):

@@ -27,7 +27,7 @@ LIB = os.path.join(PKG, "libpkv.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 SOURCES = ["api.cu", "planner.cpp", "prefill_sm100.cu", "decode_sm100.cu", "merge.cu", "mla_sm100.cu", "mla_decode_sm100.cu",
-           "decode_noalloc.cu", "append.cu", "selftest.cu", "decode_fp8_sm100.cu"]
+           "decode_noalloc.cu", "append.cu", "selftest.cu", "decode_fp8_sm100.cu", "kv_fp8_expand.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", CSRC, "-I", INCLUDE]

@@ -14,7 +14,9 @@
 
 namespace pkv {
 cudaError_t launch_prefill(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
-                           const void*, int32_t, void*, float*, cudaStream_t);
+                           const void*, int32_t, void*, float*, const float*, const float*, cudaStream_t);
+cudaError_t launch_kv_fp8_expand(const LaunchGeom&, const DeviceView&, const int32_t*, int32_t, const void*,
+                                 const void*, void*, void*, int32_t*, cudaStream_t);
 cudaError_t launch_decode(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
                           const void*, void*, float*, cudaStream_t);
 cudaError_t launch_mla(const LaunchGeom&, const DeviceView&, const int32_t*, const void*, const void*,
@@ -38,7 +40,10 @@ struct pkv_plan {
   const int32_t* kv_indices = nullptr;  // device, borrowed
   // workspace layout (byte offsets)
   size_t off_status = 0, off_units = 0, off_merges = 0, off_reqs = 0, off_cta = 0, off_row0 = 0, off_lse = 0, off_o = 0,
-         off_packed = 0, total = 0;
+         off_packed = 0, off_fp8_k = 0, off_fp8_v = 0, off_fp8_idx = 0, total = 0;
+  bool kv_fp8 = false;          // planned for pkv_run_fp8_kv (kv_fp8 option)
+  uint8_t* ws = nullptr;        // device workspace (set by pkv_plan_upload)
+  int32_t page_entries = 0;     // kv_indptr[batch]: entries of the page table
   size_t staging_bytes = 0;
   void* staging = nullptr;  // host copy of [status | units | merges | reqs | cta_ptr]
   bool staging_pinned = false;
@@ -89,6 +94,18 @@ void layout_workspace(pkv_plan* p) {
   p->off_packed = off;
   if (s.kind == kKindMla)  // the packed latent copy, ckv | kpe per key (at least one row for the tensor map)
     off = align256(off + (size_t)std::max(1, s.geom.packed_rows) * (s.geom.head_dim + s.geom.head_dim_pe) * 2);
+  // prefill over an FP8 cache: bf16 copies of the batch's K and V pages
+  // ([entries][page_size][Hk][D]) and their identity page table
+  const size_t fp8_page_bytes =
+      p->kv_fp8 && s.kind == kKindPrefill
+          ? (size_t)s.geom.page_size * s.geom.num_kv_heads * s.geom.head_dim * 2 : 0;
+  const size_t fp8_entries = fp8_page_bytes ? (size_t)std::max(1, p->page_entries) : 0;
+  p->off_fp8_k = off;
+  off = align256(off + fp8_entries * fp8_page_bytes);
+  p->off_fp8_v = off;
+  off = align256(off + fp8_entries * fp8_page_bytes);
+  p->off_fp8_idx = off;
+  off = align256(off + fp8_entries * sizeof(int32_t));
   p->total = off;
 }
 
@@ -104,6 +121,8 @@ pkv_status create_common(const PlanInput& in, const int32_t* kv_indices, pkv_pla
     return fail(rc == 1 ? PKV_EINVAL : PKV_EUNSUPPORTED, err);
   }
   p->kv_indices = kv_indices;
+  p->kv_fp8 = in.kv_fp8 != 0;
+  p->page_entries = in.batch > 0 ? in.kv_indptr[in.batch] : 0;
   layout_workspace(p);
   *out = p;
   return PKV_OK;
@@ -202,6 +221,7 @@ pkv_status pkv_plan_upload(pkv_plan* p, void* workspace, size_t bytes, void* str
   p->dv.cta_ptr = reinterpret_cast<const int32_t*>(d + p->off_cta);
   p->dv.kv_row0 = reinterpret_cast<const int32_t*>(d + p->off_row0);
   p->dv.packed = d + p->off_packed;
+  p->ws = d;
   p->uploaded = true;
   return PKV_OK;
 }
@@ -220,7 +240,8 @@ pkv_status pkv_run(const pkv_plan* p, const void* q, const void* k_cache, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = s.kind == kKindDecode
                       ? launch_decode(s.geom, p->dv, p->kv_indices, q, k_cache, v_cache, o, lse, st)
-                      : launch_prefill(s.geom, p->dv, p->kv_indices, q, k_cache, v_cache, num_pages, o, lse, st);
+                      : launch_prefill(s.geom, p->dv, p->kv_indices, q, k_cache, v_cache, num_pages, o, lse,
+                                       nullptr, nullptr, st);
   if (e == cudaSuccess) e = launch_merge_tasks(s.geom, p->dv, o, lse, st);
   if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
   return PKV_OK;
@@ -252,8 +273,10 @@ pkv_status pkv_run_fp8_kv(const pkv_plan* p, const void* q, const void* k_codes,
                           void* stream) {
   if (!p) return fail(PKV_EINVAL, "plan is NULL");
   const Schedule& s = p->sched;
-  if (s.kind != kKindDecode)
-    return fail(PKV_EUNSUPPORTED, "FP8 KV cache: decode plans only (every qo_len <= 1, group <= 16)");
+  if (s.kind != kKindDecode && s.kind != kKindPrefill) return fail(PKV_EINVAL, "MLA plan: FP8 KV cache is GQA/MHA only");
+  if (s.kind == kKindPrefill && !p->kv_fp8)
+    return fail(PKV_EUNSUPPORTED, "FP8 KV cache with a prefill plan: create the plan with pkv_plan_options.kv_fp8 = 1 "
+                                  "(it reserves the workspace for the bf16 copy of the pages)");
   if (s.geom.kv_layout != 0) return fail(PKV_EUNSUPPORTED, "FP8 KV cache: NHD pages only");
   if (s.geom.head_dim != 64 && s.geom.head_dim != 128)
     return fail(PKV_EUNSUPPORTED, "FP8 KV cache: head_dim 64 or 128");
@@ -264,7 +287,19 @@ pkv_status pkv_run_fp8_kv(const pkv_plan* p, const void* q, const void* k_codes,
     return fail(PKV_EINVAL, "tensor pointers must be 16-byte aligned");
   if (num_pages <= 0) return fail(PKV_EINVAL, "num_pages must be positive");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_decode_fp8(s.geom, p->dv, p->kv_indices, q, k_codes, v_codes, k_scale, v_scale, o, lse, st);
+  cudaError_t e = cudaSuccess;
+  if (s.kind == kKindDecode) {
+    e = launch_decode_fp8(s.geom, p->dv, p->kv_indices, q, k_codes, v_codes, k_scale, v_scale, o, lse, st);
+  } else {
+    // the batch's pages as bf16 in the workspace, then the tensor-core prefill on
+    // that copy through an identity page table, the scales applied per kv head
+    void* kc = p->ws + p->off_fp8_k;
+    void* vc = p->ws + p->off_fp8_v;
+    int32_t* idx = reinterpret_cast<int32_t*>(p->ws + p->off_fp8_idx);
+    e = launch_kv_fp8_expand(s.geom, p->dv, p->kv_indices, p->page_entries, k_codes, v_codes, kc, vc, idx, st);
+    if (e == cudaSuccess)
+      e = launch_prefill(s.geom, p->dv, idx, q, kc, vc, std::max(1, p->page_entries), o, lse, k_scale, v_scale, st);
+  }
   if (e == cudaSuccess) e = launch_merge_tasks(s.geom, p->dv, o, lse, st);
   if (e != cudaSuccess) return fail(PKV_ECUDA, std::string("launch: ") + cudaGetErrorString(e));
   return PKV_OK;

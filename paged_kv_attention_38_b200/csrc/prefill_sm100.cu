@@ -109,6 +109,11 @@ struct Args {
   int32_t q_tma;      // Q tiles by TMA (group divides 128) or by cp.async
   int32_t kv_tma;     // K/V pages by TMA (page_size >= 8; the kRows = false instance) or by cp.async rows
   int32_t oob_row;    // a pool row index past the end: TMA zero-fills it
+  // Per-kv-head scales of a quantised cache whose values were expanded to bf16
+  // codes (NULL: 1), read by the kScaled instances only: K's multiplies the
+  // scores, V's the output.
+  const float* k_scale;
+  const float* v_scale;
 };
 
 // kRows: K/V arrive as single rows by cp.async (page_size < 8) instead of whole
@@ -120,7 +125,7 @@ struct Args {
 // units with keys), so the producer streams the next unit's Q and K/V and the
 // tensor core starts its first QK^T while the softmax warps still write the
 // previous unit's output.
-template <int D, bool kRows, bool kHnd>
+template <int D, bool kRows, bool kHnd, bool kScaled>
 __global__ void __launch_bounds__(kThreadsOf<kRows>, 1) prefill_kernel(const __grid_constant__ Args a) {
   constexpr int kProdThreads = kProdThreadsOf<kRows>;
   constexpr int kRegsSupport = kRegsSupportOf<kRows>;
@@ -426,7 +431,7 @@ __global__ void __launch_bounds__(kThreadsOf<kRows>, 1) prefill_kernel(const __g
     const int ti = warp >> 2;          // query tile
     const int r = tid & (kTileM - 1);  // row in tile == TMEM lane
     const int ru = ti * kTileM + r;    // row in unit
-    const float scale = a.g.sm_scale_log2;
+    const float scale0 = a.g.sm_scale_log2;
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t s_tm = lane_base + ti * kBlockN;
     const uint32_t o_tm = lane_base + 256 + ti * 128;
@@ -435,9 +440,13 @@ __global__ void __launch_bounds__(kThreadsOf<kRows>, 1) prefill_kernel(const __g
       // Only what the KV loop needs stays live across it; the epilogue reads
       // the unit again (the softmax warps run close to their register budget).
       int n_tiles, kv_lo, limit;
+      float scale = scale0;  // base-2 score scale (times this unit's kv-head K scale)
       {
         const WorkUnit unit = a.dv.units[ui];
         const ReqInfo req = a.dv.reqs[unit.req];
+        if constexpr (kScaled) {
+          if (a.k_scale) scale *= a.k_scale[unit.kv_head];
+        }
         n_tiles = tiles_of(unit);
         kv_lo = unit.kv_lo;
         const int t = (unit.row0 + (ru < unit.rows ? ru : 0)) / G;
@@ -530,7 +539,10 @@ __global__ void __launch_bounds__(kThreadsOf<kRows>, 1) prefill_kernel(const __g
       const ReqInfo req = a.dv.reqs[unit.req];
       const bool row_ok = ru < unit.rows;
       const int pr = unit.row0 + (row_ok ? ru : 0);
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      float inv_l = l > 0.f ? 1.f / l : 0.f;
+      if constexpr (kScaled) {
+        if (a.v_scale) inv_l *= a.v_scale[unit.kv_head];
+      }
       const float lse2 = l > 0.f ? m + __log2f(l) : -INFINITY;
       const int tok = req.q_start + pr / G;
       const int h = unit.kv_head * G + pr % G;
@@ -696,20 +708,27 @@ bool make_map(CUtensorMap* m, const void* base, int D, int heads, int64_t rows, 
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool kRows, bool kHnd>
+template <int D, bool kRows, bool kHnd, bool kScaled = false>
 cudaError_t launch_as(const Args& a, cudaStream_t stream) {
   const size_t smem = sizeof(Smem<D>) + 1024;
   static std::atomic<uint64_t> configured{0};
-  cudaError_t e = set_smem_attrs_once((const void*)prefill_kernel<D, kRows, kHnd>, (int)smem, configured, false);
+  cudaError_t e =
+      set_smem_attrs_once((const void*)prefill_kernel<D, kRows, kHnd, kScaled>, (int)smem, configured, false);
   if (e != cudaSuccess) return e;
-  prefill_kernel<D, kRows, kHnd><<<a.g.num_ctas, kThreadsOf<kRows>, smem, stream>>>(a);
+  prefill_kernel<D, kRows, kHnd, kScaled><<<a.g.num_ctas, kThreadsOf<kRows>, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
 // One instance per K/V path and page layout, so that each holds only its own
-// address arithmetic (the NHD instances are unchanged by the HND ones).
+// address arithmetic (the NHD instances are unchanged by the HND ones), and
+// NHD instances with per-kv-head scales for the expanded FP8 cache (the bf16
+// instances carry none of that code).
 template <int D>
 cudaError_t launch(const Args& a, cudaStream_t stream) {
+  if (a.k_scale || a.v_scale) {
+    if (a.g.kv_layout == 1) return cudaErrorInvalidValue;
+    return a.kv_tma ? launch_as<D, false, false, true>(a, stream) : launch_as<D, true, false, true>(a, stream);
+  }
   if (a.g.kv_layout == 1)
     return a.kv_tma ? launch_as<D, false, true>(a, stream) : launch_as<D, true, true>(a, stream);
   return a.kv_tma ? launch_as<D, false, false>(a, stream) : launch_as<D, true, false>(a, stream);
@@ -719,9 +738,11 @@ cudaError_t launch(const Args& a, cudaStream_t stream) {
 
 cudaError_t launch_prefill(const LaunchGeom& g, const DeviceView& dv, const int32_t* kv_indices, const void* q,
                            const void* k, const void* v, int32_t num_pages, void* o, float* lse,
-                           cudaStream_t stream) {
+                           const float* k_scale, const float* v_scale, cudaStream_t stream) {
   if (g.num_units == 0 || g.num_ctas == 0) return cudaSuccess;
   Args a{};
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k = static_cast<const __nv_bfloat16*>(k);
   a.v = static_cast<const __nv_bfloat16*>(v);

@@ -367,9 +367,9 @@ def test_fp8_kv_workload_and_host_checks():
 
 
 def test_fp8_kv_entry_rejects_unsupported_plans():
-    """pkv_run_fp8_kv refuses prefill plans and HND decode plans with
-    PKV_EUNSUPPORTED before touching any pointer, and a decode plan that was
-    never uploaded with PKV_EINVAL."""
+    """pkv_run_fp8_kv refuses prefill plans made without the kv_fp8 option and
+    HND plans with PKV_EUNSUPPORTED before touching any pointer, and plans that
+    were never uploaded with PKV_EINVAL."""
     lib = pkv.load_library()
     args = [None] * 5 + [1, None, None, None]
 
@@ -380,9 +380,27 @@ def test_fp8_kv_entry_rejects_unsupported_plans():
     pre = _plan(W.tiny_prefill())
     assert pre.kind == pkv.KIND_PREFILL
     st, msg = call(pre)
-    assert st == 2 and "decode plans only" in msg
+    assert st == 2 and "kv_fp8" in msg
+    st, msg = call(_plan(W.tiny_prefill(), kv_fp8=True))
+    assert st == 1 and "not uploaded" in msg
     dec = _lengths_problem([1, 1], [300, 40], hq=8, hk=2, d=128, ps=16, causal=False)
     st, msg = call(_plan(dec, kv_layout=1))
     assert st == 2 and "NHD" in msg
     st, msg = call(_plan(dec))
     assert st == 1 and "not uploaded" in msg
+
+
+def test_fp8_prefill_plan_reserves_page_copy():
+    """A prefill plan made with kv_fp8 reserves the bf16 copy of the batch's K and
+    V pages ([entries][page_size][Hk][D]) and its identity page table in the
+    workspace; a decode plan and an MLA plan reserve nothing for it."""
+    def align(x):
+        return (x + 255) // 256 * 256
+
+    p = _lengths_problem([30, 0, 70], [100, 17, 70], hq=8, hk=2, d=64, ps=16, causal=True)
+    entries = int(p.kv_indptr[-1])
+    base, fp8 = _plan(p).workspace_bytes, _plan(p, kv_fp8=True).workspace_bytes
+    page = 16 * 2 * 64 * 2
+    assert fp8 - base == 2 * align(entries * page) + align(4 * entries)
+    dec = _lengths_problem([1, 1], [300, 40], hq=8, hk=2, d=128, ps=16, causal=False)
+    assert _plan(dec, kv_fp8=True).workspace_bytes == _plan(dec).workspace_bytes

@@ -320,13 +320,49 @@ def test_fp8_kv_decode_query_range(qmul):
         assert_parity(o, lse, o_ref, l_ref, what=f"fp8 q x {qmul}")
 
 
-def test_fp8_kv_rejects_prefill_plan():
+def test_fp8_kv_prefill_needs_kv_fp8_plan():
     p = W.make_fp8_kv_problem("fp8pre", [4, 2], [40, 9], num_qo_heads=4, num_kv_heads=2, head_dim=128,
-                              page_size=16, seed=4)
+                              page_size=16, seed=4, causal=True)
     d = to_dev(p)
     pl = pkv.plan(p.qo_indptr, p.kv_indptr, d["kv_indices"], p.kv_last_page_len, 4, 2, 128, 16, True, p.sm_scale)
-    with pytest.raises(Exception, match="decode plans only"):
+    with pytest.raises(Exception, match="kv_fp8"):
         pkv.run_fp8_kv(pl, d["q"], d["k_cache"], d["v_cache"])
+
+
+FP8_PREFILL = [
+    # qo_lens, kv_lens, hq, hk, d, page, causal, forced kv chunk (0 = planner's)
+    ([70, 200], [70, 200], 8, 2, 128, 16, True, 0),        # page TMA path, causal GQA
+    ([90, 33], [150, 33], 16, 1, 64, 1, True, 0),          # row gather, chunked prefill (qo < kv)
+    ([45, 160], [300, 160], 8, 8, 128, 64, False, 128),    # MHA, non-causal, split KV
+    ([100, 0, 64], [100, 20, 0], 12, 4, 128, 16, True, 0), # group 3 (cp.async Q), no queries / no keys
+]
+
+
+@pytest.mark.parametrize("case", FP8_PREFILL, ids=lambda c: f"h{c[2]}_{c[3]}_d{c[4]}_p{c[5]}_c{int(c[6])}_k{c[7]}")
+def test_fp8_kv_prefill(case):
+    """Prefill over the FP8 cache: the pages expanded to bf16 in the workspace, the
+    tensor-core prefill on the copy with the per-head scales applied."""
+    qo, kv, hq, hk, d, ps, causal, chunk = case
+    p = W.make_fp8_kv_problem("fp8pre", qo, kv, num_qo_heads=hq, num_kv_heads=hk, head_dim=d, page_size=ps,
+                              seed=zlib.crc32(str(case).encode()) % 10000, causal=causal)
+    o, lse, pl = gpu_run_fp8(p, **({"kv_chunk": chunk} if chunk else {}))
+    assert pl.kind == pkv.KIND_PREFILL
+    if chunk:
+        assert pl.num_merges > 0
+    assert_parity(o, lse, *oracle_fp8(p), what=f"fp8 prefill {case}")
+
+
+@pytest.mark.parametrize("qo", [[60, 1], [1, 1]], ids=["prefill", "decode"])
+def test_fp8_kv_nan_codes_outside_the_keys(qo):
+    """NaN codes in slots past a request's last key (in its last page and in pages
+    no request lists) never reach the output."""
+    p = W.make_fp8_kv_problem("fp8nan", qo, [60, 37], num_qo_heads=8, num_kv_heads=2, head_dim=128, page_size=16,
+                              seed=21, causal=qo[0] > 1, pool_pages=12)
+    valid = W._valid_slot_mask(p.kv_indptr, p.kv_indices, p.kv_last_page_len, p.page_size, p.num_pages)
+    p.k_cache[~valid] = 0x7F
+    p.v_cache[~valid] = 0xFF
+    o, lse, _ = gpu_run_fp8(p)
+    assert_parity(o, lse, *oracle_fp8(p), what=f"fp8 nan slots {qo}")
 
 
 @pytest.mark.slow
