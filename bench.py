@@ -100,6 +100,7 @@ def decode_bytes(p: W.PagedProblem) -> float:
 PREFILL_SOURCES = ("prefill_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
 DECODE_SOURCES = ("decode_sm100.cu", "decode_core.cuh", "sm100_ptx.cuh", "pkv_internal.h")
 DECODE_FP8_SOURCES = ("decode_fp8_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
+PREFILL_FP8_SOURCES = ("prefill_sm100.cu", "kv_fp8_expand.cu", "sm100_ptx.cuh", "pkv_internal.h")
 MLA_SOURCES = ("mla_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
 MLA_DECODE_SOURCES = ("mla_decode_sm100.cu", "sm100_ptx.cuh", "pkv_internal.h")
 APPEND_SOURCES = ("append.cu",)
@@ -508,6 +509,9 @@ def run_ours(args):
     fdec = Case(W.paged_decode_fp8(shard=rank), device)
     fdec_med, fdec_ms_local = time_case(fdec, flush, extra_steps, 3)
     fdec_ms = max_over_ranks(fdec_ms_local, world)
+    pfp8 = Case(W.gqa_prefill_fp8(shard=rank), device)
+    pfp8_med, pfp8_ms_local = time_case(pfp8, flush, extra_steps, 3)
+    pfp8_ms = max_over_ranks(pfp8_ms_local, world)
     app = AppendCase(W.gqa_prefill(shard=rank), device)
     app_med, app_ms_local = time_case(app, flush, extra_steps, 3)
     app_ms = max_over_ranks(app_ms_local, world)
@@ -551,6 +555,12 @@ def run_ours(args):
         "traffic": profiled_traffic("decode_fp8_b32_h32_kv8_d128_ps16.md", DECODE_FP8_SOURCES,
                                     kv_tokens=int(fdec.p.kv_lens.sum())),
         "ms": round(fdec_ms, 4), "in_step": False}
+    pfp8_tf = attention_flops(pfp8.p) / (pfp8_ms * 1e-3) / 1e12
+    roofs["prefill_kernel<128> over an FP8 E4M3 KV cache (h16/kv1/d128/ps64; expand + prefill)"] = {
+        "bound": "tensor", "achieved": round(pfp8_tf, 2), "peak": peak_burst, "unit": "TFLOP/s",
+        "frac": round(pfp8_tf / peak_burst, 4),
+        "traffic": profiled_traffic("prefill_fp8_h16_kv1_d128_ps64.md", PREFILL_FP8_SOURCES),
+        "ms": round(pfp8_ms, 4), "in_step": False}
     app_gbs = app.bytes / (app_ms * 1e-3) / 1e9
     roofs["append_kernel (h16/kv1/d128/ps64 batch)"] = {
         "bound": "hbm", "achieved": round(app_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(app_gbs / hbm, 4),
@@ -614,6 +624,12 @@ def run_ours(args):
                           "workload": "paged_decode_b128_h32_kv8_d128_ps16 over an FP8 E4M3 KV cache with "
                                       "per-kv-head scales, kv_len U[1024,8192]",
                           "timed": "alone, outside the step, L2 flushed before each launch"}
+    line["prefill_fp8"] = {"value": round(pfp8_tf, 2), "unit": "TFLOP/s", "ms": round(pfp8_ms, 4),
+                           "flops": attention_flops(pfp8.p), "units": pfp8.plan.num_units,
+                           "workload": "the config-2 prefill batch (h16/kv1/d128/ps64, causal, U[512,4096]) over "
+                                       "an FP8 E4M3 KV cache with per-kv-head scales; the pages expanded to bf16, "
+                                       "then the tensor-core prefill",
+                           "timed": "alone, outside the step, L2 flushed before each launch pair"}
     line["append"] = {"value": round(app_gbs, 1), "unit": "GB/s", "ms": round(app_ms, 4), "bytes": app.bytes,
                       "rows": app.nnz, "workload": "append of the whole h16/kv1/d128/ps64 prefill batch (K and V)",
                       "timed": "alone, outside the step, L2 flushed before each launch"}
@@ -631,7 +647,7 @@ def run_only(args, device, flush):
               "sparse": lambda: W.sparse_vs_dense(16, 2048, False),
               "dense": lambda: W.sparse_vs_dense(16, 2048, True),
               "mla_decode": W.mla_decode, "decode_fp8": W.paged_decode_fp8,
-              "decode_fp8_small": lambda: W.paged_decode_fp8(batch=32)}
+              "decode_fp8_small": lambda: W.paged_decode_fp8(batch=32), "prefill_fp8": W.gqa_prefill_fp8}
     if args.only == "append":
         c = AppendCase(W.gqa_prefill(), device)
         sampler = ClockSampler(device.index or 0)
@@ -740,7 +756,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the vector-sparse vs dense sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["prefill", "decode", "decode_small", "mla", "mla_decode", "sparse", "dense", "append",
-                                       "decode_fp8", "decode_fp8_small"], default=None,
+                                       "decode_fp8", "decode_fp8_small", "prefill_fp8"], default=None,
                     help="time one workload alone (profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

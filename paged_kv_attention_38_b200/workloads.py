@@ -277,6 +277,15 @@ def gqa_prefill(batch: int = 8, lo: int = 512, hi: int = 4096, shard: int = 0) -
                         causal=True, seed=seed)
 
 
+def gqa_prefill_fp8(batch: int = 8, lo: int = 512, hi: int = 4096, shard: int = 0) -> PagedProblem:
+    """The causal GQA prefill batch of ``gqa_prefill`` (same lengths, h16/kv1/d128/ps64)
+    over a per-head-scale FP8 E4M3 KV cache."""
+    seed = SEED_BASE + 2 + 10000 * shard
+    lens = uniform_lengths(batch, lo, hi, _gen(seed + 7))
+    return make_fp8_kv_problem("gqa_paged_prefill_fp8kv_h16_kv1_d128_ps64", lens, lens, num_qo_heads=16,
+                               num_kv_heads=1, head_dim=128, page_size=64, seed=seed + 900, causal=True)
+
+
 SPARSE_DENSE_SWEEP = [(1, 512), (1, 2048), (1, 8192), (16, 512), (16, 2048), (16, 8192),
                       (64, 512), (64, 2048)]
 

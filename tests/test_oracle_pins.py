@@ -426,6 +426,9 @@ def test_workload_shapes():
     assert g.batch == 8 and g.q.shape[1:] == (16, 128) and g.page_size == 64
     assert np.all((g.qo_lens >= 512) & (g.qo_lens <= 4096))
     assert sorted(g.kv_indices.tolist()) == list(range(g.num_pages))
+    f = W.gqa_prefill_fp8()
+    assert f.is_fp8_kv and f.causal and list(f.qo_lens) == list(g.qo_lens) and list(f.kv_lens) == list(g.kv_lens)
+    assert f.k_cache.dtype == torch.uint8 and f.k_cache.shape[1:] == (64, 1, 128)
 
 
 # ---------------------------------------------------------------------------
