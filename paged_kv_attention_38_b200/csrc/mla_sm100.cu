@@ -115,6 +115,9 @@ struct PackArgs {
 // 1152-byte row as 72 16-byte pieces, the loads of its four rows first.
 constexpr int kPackKeys = 32;
 __global__ void __launch_bounds__(256) mla_pack_kernel(const __grid_constant__ PackArgs a) {
+  // the attention kernel may start now: it waits for this grid before its
+  // first read of the packed rows (programmatic dependent launch)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int P = a.page_size, shift = a.page_shift;
   for (int b = blockIdx.y; b < a.batch; b += gridDim.y) {
@@ -222,6 +225,13 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(const __grid_constant_
           tma_prefetch_l2_2d(&a.tm_qpe, 0, nrow);
         }
         const int krow0 = a.dv.kv_row0[unit.req] + unit.kv_lo;
+        if (g == 0) {
+          // The kernel is launched as a programmatic dependent of the pack
+          // kernel: everything above overlaps it, the packed rows are read only
+          // after it has completed and its writes are visible.
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
         for (int j = 0; j < n_tiles; ++j, ++g) {
           const int st = g % kStages;
           if (g >= kStages) mbar_wait(&sm.kv_empty[st], ((g / kStages) - 1) & 1, wc);
@@ -520,7 +530,22 @@ cudaError_t launch_mla(const LaunchGeom& g, const DeviceView& dv, const int32_t*
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = set_smem_attrs_once((const void*)mla_kernel, (int)smem, g_configured, false);
   if (e != cudaSuccess) return e;
-  mla_kernel<<<g.num_ctas, kThreads, smem, stream>>>(a);
+  // Programmatic dependent launch of the pack kernel: CTAs may start while it
+  // runs (they read Q and the plan, both complete before it started, and wait
+  // for it before the packed rows). Without a pack launch the previous kernel
+  // on the stream is the caller's, so the launch is an ordinary one.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)g.num_ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g.packed_rows > 0 ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, mla_kernel, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
