@@ -247,7 +247,12 @@ class Case:
 
     @property
     def launches(self) -> int:
-        return 1 + (1 if self.plan.num_merges > 0 else 0)
+        n = 1 + (1 if self.plan.num_merges > 0 else 0)  # the attention kernel and its split-KV merge
+        if self.plan.kind == pkv.KIND_MLA:
+            n += 1  # the latent rows packed before the MLA prefill kernel
+        if self.p.is_fp8_kv and self.plan.kind == pkv.KIND_PREFILL:
+            n += 1  # the FP8 pages expanded to bf16 before the prefill kernel
+        return n
 
     def run(self):
         if self.p.is_mla:
